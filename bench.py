@@ -1,0 +1,427 @@
+"""Benchmark of the expert-balance hot path on B200.
+
+One step = one pass of the whole path over one microbatch of one layer of the
+Qwen3-235B-A22B-shaped workload (R=32 simulated EP ranks, E=128, top-8,
+8192 tokens/rank, hidden 4096, 1 redundant slot/rank, min quota 1024):
+ep_balance_layer (load matrix, quota solve, local-first rerouting, token rows)
+-> ep_stage_replicas (replica weights into the shared slots)
+-> ep_dispatch_layout (bf16 token rows into per-instance contiguous buffers).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Multi-GPU: the path does not shard, so N ranks run N independent replicas of
+the workload (weak scaling, no data collective); time = max over ranks.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("µs per layer balance+dispatch plan; routed tokens/s; permute GB/s vs HBM peak; "
+          "max/mean load")
+UNIT = "routed tokens/s"
+L2_BYTES = 126 * 2**20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel, workload):
+    """dram bytes per launch from the committed ncu summary, if the kernel source
+    is unchanged since the capture; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}:{workload}")
+    if not e or e.get("source_sha") != _source_hash(e.get("sources", [])):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.index = str(device_index)
+        try:  # address the GPU by PCI bus id: visible-device indices need not match
+            import torch
+
+            pr = torch.cuda.get_device_properties(device_index)
+            self.index = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+        except Exception:
+            pass
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ep_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        sm = sorted(r[0] for r in loaded)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(loaded)}
+
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_gpu(args):
+    import datetime
+
+    import numpy as np
+    import torch
+
+    from moe_expert_load_b200 import Plan, config_from_workload
+    from workloads import get_config, topk_ids
+
+    world, rank, local = _dist_init()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = get_config(args.workload)
+    if w.layers > 1:
+        w = w.replace(layers=1)
+    dev = torch.device("cuda", local)
+    ids_np = topk_ids(w)
+    ids = torch.from_numpy(ids_np).to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    hidden = torch.randn((w.N, w.hidden), generator=g, device=dev).to(torch.bfloat16)
+    native_w = torch.randn((w.E, w.expert_elems), generator=g, device=dev).to(torch.bfloat16)
+    slots = torch.zeros((w.R, w.S, w.expert_elems), dtype=torch.bfloat16, device=dev)
+    rows_cap = w.A + (w.N if w.shared_expert else 0)
+    out = torch.empty((rows_cap, w.hidden), dtype=torch.bfloat16, device=dev)
+    plan = Plan(config_from_workload(w, num_layers=1), device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        plan.balance_layer(0, ids)
+        plan.stage_replicas(0, native_w, slots)
+        if ev is not None:
+            ev[0].record(stream)
+        plan.dispatch_layout(0, hidden, out=out)
+        if ev is not None:
+            ev[1].record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    stats = plan.read_layer_stats(0)
+    launches_per_step = (4 + (3 if w.shared_expert else 1)) + 1 + 1  # balance + stage + dispatch
+
+    # ---- timed region: K whole steps --------------------------------------
+    perm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for k in range(args.steps):
+            step(perm_ev[k])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms_total = t0.elapsed_time(t1)
+    if dist is not None:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    perm_ms = [a.elapsed_time(b) for a, b in perm_ev]
+    perm_avg_ms = sum(perm_ms) / len(perm_ms)
+
+    # ---- plan latency alone, with L2 flushed before every call -------------
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    plan_us = []
+    for k in range(args.plan_iters + 3):
+        flush.fill_(k & 0xFF)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        plan.balance_layer(0, ids)
+        b.record(stream)
+        b.synchronize()
+        if k >= 3:
+            plan_us.append(a.elapsed_time(b) * 1e3)
+    plan_us.sort()
+
+    # ---- staging alone ------------------------------------------------------
+    stage_ms = []
+    for k in range(6):
+        flush.fill_(k)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        plan.stage_replicas(0, native_w, slots)
+        b.record(stream)
+        b.synchronize()
+        if k >= 1:
+            stage_ms.append(a.elapsed_time(b))
+    n_rep = int(stats["replicas"])
+    view = plan.view(0)
+    rep_ptr = view["replica_expert_ptr"].cpu().numpy()
+    n_rep_exp = int((np.diff(rep_ptr) > 0).sum())
+    stage_bytes = (n_rep_exp + n_rep) * w.expert_elems * 2
+    stage_gbs = stage_bytes / (sum(stage_ms) / len(stage_ms) * 1e-3) / 1e9 if n_rep else 0.0
+
+    # ---- end to end through the public API with host buffers ---------------
+    e2e = None
+    if args.e2e_steps > 0:
+        ids_h = torch.from_numpy(ids_np).pin_memory()
+        hidden_h = hidden.cpu().pin_memory()
+        e2e_ms = []
+        for k in range(args.e2e_steps + 1):
+            barrier()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ids.copy_(ids_h, non_blocking=True)
+            hidden.copy_(hidden_h, non_blocking=True)
+            plan.balance_layer(0, ids)
+            plan.stage_replicas(0, native_w, slots)
+            plan.dispatch_layout(0, hidden, out=out)
+            st = plan.read_layer_stats(0)  # device -> host read of the step's result
+            b.record(stream)
+            b.synchronize()
+            if k >= 1:
+                e2e_ms.append(a.elapsed_time(b))
+        e2e_step = sum(e2e_ms) / len(e2e_ms)
+        if dist is not None:
+            tt = torch.tensor([e2e_step], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_step = float(tt.item())
+        e2e = {"value": world * w.A / (e2e_step * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": int(ids_np.nbytes + hidden.numel() * 2),
+               "d2h_bytes_per_step": 64, "steps": args.e2e_steps, "ms_per_step": e2e_step}
+        assert st["rows"] == stats["rows"]
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    peak, peak_kind = _peaks()
+    perm_bytes = (w.N + rows_cap) * w.hidden * 2  # each token row read once, written per row
+    achieved = perm_bytes / (perm_avg_ms * 1e-3) / 1e9
+    traffic = _traffic("k_permute", w.name)
+    A = int(stats["assignments"])
+    line = {
+        "metric": METRIC,
+        "value": world * A / (ms_step * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int32",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{w.name}: Qwen3-235B-A22B-shaped MoE layer, R={w.R} simulated EP ranks, "
+                        f"E={w.E}, top-{w.K}, T={w.T} tokens/rank, hidden {w.hidden} bf16, "
+                        f"S={w.S} slot/rank of 3x{w.hidden}x{w.ffn} bf16, m={w.m}, Zipf s={w.zipf_s}",
+            "step": "ep_balance_layer + ep_stage_replicas + ep_dispatch_layout",
+            "l2": "inputs larger than L2: each step's dispatch writes "
+                  f"{rows_cap * w.hidden * 2 / 1e9:.1f} GB, evicting L2 between steps; "
+                  "plan latency measured after a 252 MiB L2 flush",
+            "parallelism": f"replicas x{world} (path does not shard)",
+        },
+        "plan_us": {"median": plan_us[len(plan_us) // 2], "p90": plan_us[int(len(plan_us) * 0.9)],
+                    "iters": len(plan_us)},
+        "permute_gbs": achieved,
+        "stage_gbs": stage_gbs,
+        "max_mean_load": {"before": stats["before_max"] * w.R / A, "after": stats["after_max"] * w.R / A,
+                          "stop_reason": stats["stop_reason"],
+                          "tight_stop_reason": stats["tight_stop_reason"],
+                          "replicas": n_rep, "cap_idx": stats["cap_idx"]},
+        "roofline": {"bound": "hbm", "kernel": "k_permute", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes": perm_bytes,
+                     "launch_ms": perm_avg_ms},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    return line
+
+
+def cpu_baseline(w, budget_s=15.0, steps=None):
+    """The oracle, as it stands, on one host core: each step runs the full oracle
+    plan of the layer, then dispatches a fixed sample of tokens and stages a
+    fixed slice of every replica; the step time is scaled to the whole layer."""
+    import numpy as np
+
+    import oracle
+    from workloads import topk_ids
+
+    ids = topk_ids(w)
+    rng = np.random.default_rng(0)
+    sample_tokens = min(w.N, 4096)
+    n0 = w.N // 2 - sample_tokens // 2
+    hidden_rows = rng.integers(0, 2**16, size=(sample_tokens, w.hidden), dtype=np.uint16)
+    stage_elems = min(w.expert_elems, 1 << 20)
+    native_np = rng.integers(0, 2**16, size=(w.E, stage_elems), dtype=np.uint16)
+    slots = np.empty((w.R, w.S, stage_elems), np.uint16)
+    out = None
+    t_start = time.perf_counter()
+    fulls = []
+    k = 0
+    while True:
+        t0 = time.perf_counter()
+        p = oracle.plan(ids, E=w.E, S=w.S, m=w.m, J=w.J, shared_expert=w.shared_expert,
+                        seed=w.waterfill_seed, bonus_permille=w.waterfill_bonus_permille)
+        t1 = time.perf_counter()
+        if out is None:  # sized once; only the sample's rows are ever touched
+            out = np.empty((p.rows, w.hidden), np.uint16)
+            oracle.permute_range(p, hidden_rows, n0, out)
+        t2 = time.perf_counter()
+        oracle.permute_range(p, hidden_rows, n0, out)
+        t3 = time.perf_counter()
+        oracle.stage(p, native_np, slots)
+        t4 = time.perf_counter()
+        full = (t1 - t0) + (t3 - t2) * (w.N / sample_tokens) + (t4 - t3) * (w.expert_elems / stage_elems)
+        fulls.append(full)
+        k += 1
+        if steps is not None and k >= steps:
+            break
+        if steps is None and time.perf_counter() - t_start > budget_s:
+            break
+    full_s = sum(fulls) / len(fulls)
+    return {"value": p.A / full_s, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "steps": k, "s_per_step_extrapolated": full_s,
+            "sample": (f"{w.name}: full oracle plan of the layer each step; dispatch of tokens "
+                       f"[{n0}, {n0 + sample_tokens}) of {w.N} and staging of {stage_elems} of "
+                       f"{w.expert_elems} elements per replica, scaled to the whole layer; one thread")}
+
+
+def run_reference(args):
+    world, rank, _ = _dist_init()
+    if rank != 0:
+        return None
+    from workloads import get_config
+
+    w = get_config(args.workload)
+    if w.layers > 1:
+        w = w.replace(layers=1)
+    for _ in range(max(0, args.warmup)):
+        cpu_baseline(w, steps=1)
+    steps = max(1, args.steps)
+    t0 = time.perf_counter()
+    cb = cpu_baseline(w, steps=steps)
+    wall = time.perf_counter() - t0
+    return {
+        "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": cb["s_per_step_extrapolated"] * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name} (same as the CUDA arm)", "wall_s": wall},
+        "cpu_baseline": {"value": cb["value"], "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qwen")
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--plan-iters", type=int, default=100)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "cuda":
+        ap.error("--warmup must be at least 3")
+    line = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,364 @@
+// Host side of the C ABI declared in include/ep_balance.h: configuration
+// checks, the workspace layout (per-layer plan cache + shared scratch), and the
+// entry points, each of which only validates arguments and enqueues kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+cudaError_t set_plan_attributes(const Dims& d);
+cudaError_t set_copy_attributes(const Dims& d);
+}  // namespace ep
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Byte offsets of every array, relative to the workspace base.
+struct Layout {
+  // per layer (offset inside one layer block)
+  size_t load, expert_total, W0, W, inst_expert, inst_quota, inst_off, rank_base, dst_row,
+      shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, stats;
+  size_t layer_bytes;
+  // scratch (absolute)
+  size_t sub_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase;
+  size_t scratch_bytes;
+  size_t total;
+};
+
+struct Bump {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + (bytes ? bytes : 1));
+    return o;
+  }
+};
+
+ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
+  if (!c) return EP_ERR_INVALID_ARGUMENT;
+  if (c->reserved0 != 0) return EP_ERR_INVALID_ARGUMENT;
+  const int R = c->num_ranks, E = c->num_experts, K = c->top_k, T = c->tokens_per_rank;
+  if (R < 1 || E < 1 || K < 1 || T < 0 || c->slots_per_rank < 0 || c->min_replica_quota < 1 ||
+      c->num_layers < 1 || c->num_cap_candidates < 1 || c->hidden < 1 ||
+      c->expert_weight_elems < 0 || c->waterfill_bonus_permille < 0 ||
+      (c->shared_expert != 0 && c->shared_expert != 1))
+    return EP_ERR_INVALID_ARGUMENT;
+  const int Gmax = E / R + (E % R ? 1 : 0);
+  if (R > ep::kMaxR || E > ep::kMaxE || Gmax > ep::kMaxNat || K > ep::kMaxK ||
+      c->slots_per_rank > ep::kMaxS || c->num_cap_candidates > ep::kMaxJ ||
+      c->waterfill_bonus_permille > 1000 || c->hidden < 8 || (c->hidden * 2) % 16 != 0 ||
+      c->expert_weight_elems % 8 != 0)
+    return EP_ERR_UNSUPPORTED;
+  if ((int64_t)R * T * (K + 1) >= (int64_t)INT32_MAX) return EP_ERR_UNSUPPORTED;
+  // Waterfill draw weights stay below 2^32: (K + 2) * H with H <= ceil((A + N) / R) + 1
+  const int64_t H = ((int64_t)T * (K + 1) * R + R - 1) / R + 1;
+  if ((int64_t)(K + 2) * H >= ((int64_t)1 << 32)) return EP_ERR_UNSUPPORTED;
+  d->R = R;
+  d->E = E;
+  d->K = K;
+  d->T = T;
+  d->S = c->slots_per_rank;
+  d->m = c->min_replica_quota;
+  d->J = c->num_cap_candidates;
+  d->Gmax = Gmax;
+  d->sh = c->shared_expert;
+  d->G = Gmax + d->S + d->sh;
+  d->nsub = (T + ep::kSubT - 1) / ep::kSubT;
+  d->bonus = c->waterfill_bonus_permille;
+  d->hidden = c->hidden;
+  d->pad_ = 0;
+  d->seed = c->waterfill_seed;
+  d->Wn = c->expert_weight_elems;
+  return EP_OK;
+}
+
+Layout make_layout(const ep::Dims& d, int num_layers) {
+  Layout L{};
+  const size_t i4 = sizeof(int32_t);
+  Bump b;
+  L.load = b.take(i4 * d.R * d.E);
+  L.expert_total = b.take(i4 * d.E);
+  L.W0 = b.take(i4 * d.R);
+  L.W = b.take(i4 * d.R);
+  L.inst_expert = b.take(i4 * d.R * d.G);
+  L.inst_quota = b.take(i4 * d.R * d.G);
+  L.inst_off = b.take(i4 * ((size_t)d.R * d.G + 1));
+  L.rank_base = b.take(i4 * (d.R + 1));
+  L.dst_row = b.take(i4 * (size_t)d.R * d.T * d.K);
+  L.shared_rank = b.take(d.sh ? i4 * (size_t)d.R * d.T : 0);
+  L.shared_row = b.take(d.sh ? i4 * (size_t)d.R * d.T : 0);
+  L.cand = b.take(i4 * 3 * d.J);
+  L.rep_list = b.take(i4 * ((size_t)d.R * d.S + 1));
+  L.rep_eptr = b.take(i4 * (d.E + 1));
+  L.rep_nexp = b.take(i4);
+  L.rep_experts = b.take(i4 * ((size_t)d.R * d.S + 1));
+  L.stats = b.take(sizeof(ep_layer_stats));
+  L.layer_bytes = b.off;
+  Bump s;
+  s.off = L.layer_bytes * (size_t)num_layers;
+  L.sub_cnt = s.take(i4 * (size_t)d.R * d.nsub * d.E);
+  L.wsub_cnt = s.take(d.sh ? i4 * (size_t)d.R * d.R * d.nsub : 0);
+  L.seg_ptr = s.take(i4 * (size_t)d.E * (d.R + 1));
+  L.seg_ord = s.take(i4 * (size_t)d.E * 3 * d.R);
+  L.seg_rank = s.take(i4 * (size_t)d.E * 3 * d.R);
+  L.seg_rel = s.take(i4 * (size_t)d.E * 3 * d.R);
+  L.inst_rel = s.take(i4 * (size_t)d.R * d.G);
+  L.slack = s.take(i4 * d.R);
+  L.wf = s.take(i4 * 2);
+  L.sbase = s.take(i4 * d.R);
+  L.total = s.off;
+  L.scratch_bytes = s.off - L.layer_bytes * (size_t)num_layers;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+struct ep_plan {
+  ep_config cfg;
+  ep::Dims d;
+  Layout lay;
+  char* ws;
+  size_t ws_bytes;
+  int device;
+  int num_sms;
+  unsigned char* planned;  // per layer: balanced at least once
+};
+
+namespace {
+
+int32_t* at(const ep_plan* p, size_t off) { return reinterpret_cast<int32_t*>(p->ws + off); }
+
+ep::LayerBuf layer_buf(const ep_plan* p, int layer) {
+  const size_t b = p->lay.layer_bytes * (size_t)layer;
+  const Layout& l = p->lay;
+  ep::LayerBuf L;
+  L.load = at(p, b + l.load);
+  L.expert_total = at(p, b + l.expert_total);
+  L.W0 = at(p, b + l.W0);
+  L.W = at(p, b + l.W);
+  L.inst_expert = at(p, b + l.inst_expert);
+  L.inst_quota = at(p, b + l.inst_quota);
+  L.inst_off = at(p, b + l.inst_off);
+  L.rank_base = at(p, b + l.rank_base);
+  L.dst_row = at(p, b + l.dst_row);
+  L.shared_rank = p->d.sh ? at(p, b + l.shared_rank) : nullptr;
+  L.shared_row = p->d.sh ? at(p, b + l.shared_row) : nullptr;
+  L.cand = at(p, b + l.cand);
+  L.rep_list = at(p, b + l.rep_list);
+  L.rep_eptr = at(p, b + l.rep_eptr);
+  L.rep_nexp = at(p, b + l.rep_nexp);
+  L.rep_experts = at(p, b + l.rep_experts);
+  L.stats = reinterpret_cast<ep_layer_stats*>(p->ws + b + l.stats);
+  return L;
+}
+
+ep::Scratch scratch(const ep_plan* p) {
+  const Layout& l = p->lay;
+  ep::Scratch s;
+  s.sub_cnt = at(p, l.sub_cnt);
+  s.wsub_cnt = p->d.sh ? at(p, l.wsub_cnt) : nullptr;
+  s.seg_ptr = at(p, l.seg_ptr);
+  s.seg_ord = at(p, l.seg_ord);
+  s.seg_rank = at(p, l.seg_rank);
+  s.seg_rel = at(p, l.seg_rel);
+  s.inst_rel = at(p, l.inst_rel);
+  s.slack = at(p, l.slack);
+  s.wf = at(p, l.wf);
+  s.sbase = at(p, l.sbase);
+  return s;
+}
+
+ep_status_t check_layer(const ep_plan* p, int32_t layer) {
+  if (!p) return EP_ERR_INVALID_ARGUMENT;
+  if (layer < 0 || layer >= p->cfg.num_layers) return EP_ERR_INVALID_ARGUMENT;
+  return EP_OK;
+}
+
+ep_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t ep_abi_version(void) { return EP_ABI_VERSION; }
+
+const char* ep_status_string(ep_status_t s) {
+  switch (s) {
+    case EP_OK: return "ok";
+    case EP_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case EP_ERR_UNSUPPORTED: return "unsupported configuration";
+    case EP_ERR_CUDA: return "CUDA error";
+    case EP_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case EP_ERR_NOT_PLANNED: return "layer not balanced yet";
+    case EP_ERR_DEVICE_STATUS: return "device status bit set";
+    default: return "unknown status";
+  }
+}
+
+ep_status_t ep_plan_workspace_bytes(const ep_config* cfg, size_t* bytes) {
+  if (!bytes) return EP_ERR_INVALID_ARGUMENT;
+  ep::Dims d;
+  const ep_status_t st = make_dims(cfg, &d);
+  if (st != EP_OK) return st;
+  *bytes = make_layout(d, cfg->num_layers).total;
+  return EP_OK;
+}
+
+ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t workspace_bytes,
+                           ep_plan** out) {
+  if (!out || !d_workspace) return EP_ERR_INVALID_ARGUMENT;
+  *out = nullptr;
+  ep::Dims d;
+  ep_status_t st = make_dims(cfg, &d);
+  if (st != EP_OK) return st;
+  if ((reinterpret_cast<uintptr_t>(d_workspace) & (kAlign - 1)) != 0) return EP_ERR_INVALID_ARGUMENT;
+  const Layout lay = make_layout(d, cfg->num_layers);
+  if (workspace_bytes < lay.total) return EP_ERR_WORKSPACE_TOO_SMALL;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EP_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return EP_ERR_CUDA;
+  if (ep::set_plan_attributes(d) != cudaSuccess) return EP_ERR_CUDA;
+  if (ep::set_copy_attributes(d) != cudaSuccess) return EP_ERR_CUDA;
+  ep_plan* p = new (std::nothrow) ep_plan;
+  if (!p) return EP_ERR_INVALID_ARGUMENT;
+  p->planned = new (std::nothrow) unsigned char[cfg->num_layers];
+  if (!p->planned) {
+    delete p;
+    return EP_ERR_INVALID_ARGUMENT;
+  }
+  memset(p->planned, 0, (size_t)cfg->num_layers);
+  p->cfg = *cfg;
+  p->d = d;
+  p->lay = lay;
+  p->ws = static_cast<char*>(d_workspace);
+  p->ws_bytes = workspace_bytes;
+  p->device = dev;
+  p->num_sms = sms;
+  *out = p;
+  return EP_OK;
+}
+
+void ep_plan_destroy(ep_plan* plan) {
+  if (!plan) return;
+  delete[] plan->planned;
+  delete plan;
+}
+
+ep_status_t ep_balance_layer(ep_plan* plan, int32_t layer, const int32_t* d_topk_ids,
+                             void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!d_topk_ids && plan->d.T > 0) return EP_ERR_INVALID_ARGUMENT;
+  st = cuda_status(ep::launch_balance(plan->d, layer_buf(plan, layer), scratch(plan), d_topk_ids,
+                                      static_cast<cudaStream_t>(stream)));
+  if (st == EP_OK) plan->planned[layer] = 1;
+  return st;
+}
+
+ep_status_t ep_layer_view_get(const ep_plan* plan, int32_t layer, ep_layer_view* out) {
+  const ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!out) return EP_ERR_INVALID_ARGUMENT;
+  const ep::LayerBuf L = layer_buf(plan, layer);
+  out->load = L.load;
+  out->expert_total = L.expert_total;
+  out->rank_load_before = L.W0;
+  out->rank_load = L.W;
+  out->inst_expert = L.inst_expert;
+  out->inst_quota = L.inst_quota;
+  out->inst_off = L.inst_off;
+  out->rank_row_begin = L.rank_base;
+  out->dst_row = L.dst_row;
+  out->shared_rank = L.shared_rank;
+  out->shared_row = L.shared_row;
+  out->cand_max_load = L.cand;
+  out->cand_replicas = L.cand + plan->d.J;
+  out->cand_stop = L.cand + 2 * plan->d.J;
+  out->replica_list = L.rep_list;
+  out->replica_expert_ptr = L.rep_eptr;
+  out->stats = L.stats;
+  out->Gmax = plan->d.Gmax;
+  out->G = plan->d.G;
+  return EP_OK;
+}
+
+ep_status_t ep_read_layer_stats(ep_plan* plan, int32_t layer, ep_layer_stats* h_out,
+                                void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!h_out) return EP_ERR_INVALID_ARGUMENT;
+  if (!plan->planned[layer]) return EP_ERR_NOT_PLANNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ep::LayerBuf L = layer_buf(plan, layer);
+  if (cudaMemcpyAsync(h_out, L.stats, sizeof(ep_layer_stats), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return EP_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return EP_ERR_CUDA;
+  return h_out->status ? EP_ERR_DEVICE_STATUS : EP_OK;
+}
+
+ep_status_t ep_dispatch_layout(ep_plan* plan, int32_t layer, const void* d_hidden, void* d_out,
+                               int64_t out_rows_capacity, int32_t dst_rank_begin,
+                               int32_t dst_rank_end, void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!plan->planned[layer]) return EP_ERR_NOT_PLANNED;
+  if (dst_rank_begin < 0 || dst_rank_end > plan->d.R || dst_rank_begin > dst_rank_end ||
+      out_rows_capacity < 0)
+    return EP_ERR_INVALID_ARGUMENT;
+  if ((int64_t)plan->d.R * plan->d.T > 0 && (!d_hidden || !d_out)) return EP_ERR_INVALID_ARGUMENT;
+  if (!aligned16(d_hidden) || !aligned16(d_out)) return EP_ERR_INVALID_ARGUMENT;
+  if (dst_rank_begin == dst_rank_end) return EP_OK;
+  return cuda_status(ep::launch_dispatch(plan->d, layer_buf(plan, layer), d_hidden, d_out,
+                                         out_rows_capacity, dst_rank_begin, dst_rank_end,
+                                         plan->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_stage_replicas(ep_plan* plan, int32_t layer, const void* d_native_w,
+                              void* d_slots, void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!plan->planned[layer]) return EP_ERR_NOT_PLANNED;
+  if (plan->d.Wn > 0 && plan->d.S > 0 && (!d_native_w || !d_slots)) return EP_ERR_INVALID_ARGUMENT;
+  if (!aligned16(d_native_w) || !aligned16(d_slots)) return EP_ERR_INVALID_ARGUMENT;
+  return cuda_status(ep::launch_stage(plan->d, layer_buf(plan, layer), d_native_w, d_slots,
+                                      plan->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_reduce_replica_grads(ep_plan* plan, int32_t layer, void* d_slot_grads,
+                                    int32_t grad_dtype, float* d_native_grads, void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!plan->planned[layer]) return EP_ERR_NOT_PLANNED;
+  if (grad_dtype != 0 && grad_dtype != 1) return EP_ERR_INVALID_ARGUMENT;
+  if (plan->d.Wn > 0 && plan->d.S > 0 && (!d_slot_grads || !d_native_grads))
+    return EP_ERR_INVALID_ARGUMENT;
+  if (!aligned16(d_slot_grads) || !aligned16(d_native_grads)) return EP_ERR_INVALID_ARGUMENT;
+  return cuda_status(ep::launch_reduce(plan->d, layer_buf(plan, layer), d_slot_grads, grad_dtype,
+                                       d_native_grads, plan->num_sms,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_waterfill(int32_t R, int32_t T, int32_t K, const int32_t* d_load,
+                         const int32_t* d_dst_rank, uint64_t seed, int32_t bonus_permille,
+                         int32_t* d_pick, int32_t* d_count, void* stream) {
+  if (R < 1 || T < 0 || K < 0 || bonus_permille < 0) return EP_ERR_INVALID_ARGUMENT;
+  if (R > ep::kMaxR || K > ep::kMaxK || bonus_permille > 1000) return EP_ERR_UNSUPPORTED;
+  if ((int64_t)R * T * (K + 1) >= (int64_t)INT32_MAX) return EP_ERR_UNSUPPORTED;
+  if (!d_load || !d_count) return EP_ERR_INVALID_ARGUMENT;
+  if (T > 0 && (!d_pick || (K > 0 && !d_dst_rank))) return EP_ERR_INVALID_ARGUMENT;
+  return cuda_status(ep::launch_waterfill(R, T, K, d_load, d_dst_rank, seed, bonus_permille,
+                                          d_pick, d_count, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,98 @@
+// Internal definitions shared by the CUDA translation units of libep_b200.
+// Not part of the public ABI (include/ep_balance.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep_balance.h"
+
+namespace ep {
+
+constexpr int kSubT = 128;      // tokens per sub-chunk; one warp owns one sub-chunk
+constexpr int kMaxR = 128;      // ranks (4 words of 32 per warp lane)
+constexpr int kRW = 4;          // rank words per lane: lane owns ranks lane + 32*k
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 16;
+constexpr int kMaxS = 8;
+constexpr int kMaxJ = 16;
+constexpr int kMaxNat = 32;     // natives per rank: one warp lane each in the solver
+constexpr int kNoRank = 0xFF;   // "no destination" in uint8 rank buffers
+
+// Problem dimensions, passed by value to every kernel.
+struct Dims {
+  int R, E, K, T;
+  int S, m, J;
+  int Gmax, G, sh;   // natives per rank (max), columns per rank, shared column present
+  int nsub;          // sub-chunks per rank = ceil(T / kSubT)
+  int bonus;         // Waterfill local preference, permille
+  int hidden;        // bf16 elements per hidden row
+  int pad_;
+  uint64_t seed;     // Waterfill draw seed
+  int64_t Wn;        // bf16 elements per expert
+};
+
+// One layer's slot in the plan cache (all device pointers).
+struct LayerBuf {
+  int32_t* load;          // [R][E]
+  int32_t* expert_total;  // [E]
+  int32_t* W0;            // [R]
+  int32_t* W;             // [R]
+  int32_t* inst_expert;   // [R][G]
+  int32_t* inst_quota;    // [R][G]
+  int32_t* inst_off;      // [R*G+1]
+  int32_t* rank_base;     // [R+1]
+  int32_t* dst_row;       // [R][T][K]
+  int32_t* shared_rank;   // [R][T] or null
+  int32_t* shared_row;    // [R][T] or null
+  int32_t* cand;          // [3][J]: max load, replicas, stop reason
+  int32_t* rep_list;      // [R*S] slot ids grouped by expert, instance order within
+  int32_t* rep_eptr;      // [E+1]
+  int32_t* rep_nexp;      // [1] number of replicated experts
+  int32_t* rep_experts;   // [R*S] replicated experts, ascending
+  ep_layer_stats* stats;
+};
+
+// Scratch shared by all layers, reused by every balance call.
+struct Scratch {
+  int32_t* sub_cnt;   // [R][nsub][E] per-sub-chunk counts, then exclusive bases
+  int32_t* wsub_cnt;  // [R][R*nsub] shared-slot counts per (dest rank, sub-chunk), then bases
+  int32_t* seg_ptr;   // [E][R+1] first segment of each source rank, per expert
+  int32_t* seg_ord;   // [E][3R] first ordinal of the segment
+  int32_t* seg_rank;  // [E][3R] destination rank
+  int32_t* seg_rel;   // [E][3R] first row, relative to the destination rank's block
+  int32_t* inst_rel;  // [R*G] first row of an instance inside its rank's block
+  int32_t* slack;     // [R] Waterfill slack
+  int32_t* wf;        // [2] Waterfill H, B
+  int32_t* sbase;     // [R] first row of each rank's shared column
+};
+
+// ---- native placement: contiguous balanced blocks ---------------------------
+__host__ __device__ __forceinline__ int nat_count(int q, int E, int R) {
+  return E / R + (q < E % R ? 1 : 0);
+}
+__host__ __device__ __forceinline__ int nat_first(int q, int E, int R) {
+  return q * (E / R) + (q < E % R ? q : E % R);
+}
+__host__ __device__ __forceinline__ int home_of(int e, int E, int R) {
+  const int base = E / R, rem = E % R;
+  const int big = rem * (base + 1);  // experts held by the first rem ranks
+  return e < big ? e / (base + 1) : rem + (e - big) / base;
+}
+
+// ---- launchers (defined in the .cu files) ----------------------------------
+cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s,
+                           const int32_t* ids, cudaStream_t st);
+cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden, void* out,
+                            int64_t cap_rows, int rank_begin, int rank_end, int num_sms,
+                            cudaStream_t st);
+cudaError_t launch_stage(const Dims& d, const LayerBuf& L, const void* native_w, void* slots,
+                         int num_sms, cudaStream_t st);
+cudaError_t launch_reduce(const Dims& d, const LayerBuf& L, void* slot_grads, int grad_f32,
+                          float* native_grads, int num_sms, cudaStream_t st);
+cudaError_t launch_waterfill(int R, int T, int K, const int32_t* load, const int32_t* dst_rank,
+                             uint64_t seed, int bonus, int32_t* pick, int32_t* count,
+                             cudaStream_t st);
+cudaError_t set_kernel_attributes(const Dims& d);
+
+}  // namespace ep

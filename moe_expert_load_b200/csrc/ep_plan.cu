@@ -1,0 +1,944 @@
+// Balance-plan kernels for sm_100a: load matrix, quota solve, local-first
+// rerouting, token assignment and the Waterfill shared slot.
+//
+// What each kernel computes follows the UltraEP page ("300 µs to level MoE
+// expert load"): §"Getting the real load of the current layer after the Gate"
+// (global load matrix, identical deterministic solve on every rank),
+// §"Quota decides replicas and token split together" (quota per instance,
+// replica creation under S slots per rank / one instance per rank / minimum
+// quota, local instance first then remote instances by remaining quota), and
+// the Waterfill page §"Waterfill" (waterline H, slack, per-token draw).
+// Everything is integer arithmetic; all orders are fixed, so results are
+// bit-identical run to run and independent of the grid size.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kWarpsPerBlock = 8;
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the state is advanced by the
+// golden-gamma increment and finished with the variant-13 mixer.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// ---------------------------------------------------------------------------
+// a1: warp-aggregated histogram.  One warp per sub-chunk of kSubT tokens of one
+// source rank; lanes with equal ids are grouped with match.any and the group
+// leader adds the group size to the warp's private shared histogram.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, ep_layer_stats* stats) {
+  extern __shared__ int32_t sm_hist[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * kWarpsPerBlock + warp;
+  if (gw >= d.R * d.nsub) return;
+  int32_t* hist = sm_hist + warp * d.E;
+  for (int e = lane; e < d.E; e += 32) hist[e] = 0;
+  __syncwarp();
+  const int r = gw / d.nsub, sub = gw - (gw / d.nsub) * d.nsub;
+  const int t0 = sub * kSubT, t1 = min(d.T, t0 + kSubT);
+  const int32_t* src = ids + (int64_t)r * d.T * d.K;
+  const int a0 = t0 * d.K, a1 = t1 * d.K;
+  int bad = 0;
+  for (int a = a0; a < a1; a += 4 * 32) {
+    int v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = a + u * 32 + lane;
+      v[u] = idx < a1 ? __ldg(src + idx) : -1;
+      if (idx < a1 && (v[u] < 0 || v[u] >= d.E)) { bad = 1; v[u] = -1; }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const unsigned peers = __match_any_sync(kFull, v[u]);
+      if (v[u] >= 0 && lane == __ffs(peers) - 1) hist[v[u]] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  int32_t* out = s.sub_cnt + (int64_t)gw * d.E;
+  for (int e = lane; e < d.E; e += 32) out[e] = hist[e];
+  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&stats->status, EP_DEV_BAD_ID);
+}
+
+// a1 (cont.): per (source rank, expert), exclusive scan of the sub-chunk counts
+// in token order (the bases of the stable ordinals) and the load-matrix entry.
+__global__ void __launch_bounds__(256) k_scan(Dims d, Scratch s, LayerBuf L) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= d.R * d.E) return;
+  const int r = i / d.E, e = i - (i / d.E) * d.E;
+  int32_t* p = s.sub_cnt + (int64_t)r * d.nsub * d.E + e;
+  int run = 0;
+  int sub = 0;
+  for (; sub + 8 <= d.nsub; sub += 8) {
+    int c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c[u] = p[(int64_t)(sub + u) * d.E];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      p[(int64_t)(sub + u) * d.E] = run;
+      run += c[u];
+    }
+  }
+  for (; sub < d.nsub; ++sub) {
+    const int c = p[(int64_t)sub * d.E];
+    p[(int64_t)sub * d.E] = run;
+    run += c;
+  }
+  L.load[i] = run;
+}
+
+// ---------------------------------------------------------------------------
+// a2: quota solve.  One CTA; warp j runs the greedy at cap
+// C_j = ceil(A (200 + j) / (200 R)).  Greedy step: the most-loaded rank p that is
+// not stuck (smallest index on ties) gives min(max(W_p - C, m), slack_r, Q_e) of
+// its native e — natives tried by quota descending, then expert ascending, only
+// those with quota >= m — to a new replica on the rank r with the largest slack
+// C - W_r >= m among ranks with a free slot and no instance of e (smallest index
+// on ties).  If no native of p can move, p is stuck.  The run with the smallest
+// (max load, replicas, j) wins.  A lane owns ranks lane + 32k and keeps their
+// load, slot table and flags in registers; native quotas live in shared memory.
+// ---------------------------------------------------------------------------
+template <int SMAX>
+__global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scratch s) {
+  extern __shared__ int32_t sm[];
+  int32_t* Tot = sm;              // [E]
+  int32_t* Qn_all = sm + d.E;     // [J][E]
+  int32_t* cnt_e = Qn_all + d.J * d.E;  // [E+1]
+  __shared__ int32_t s_W0[kMaxR];
+  __shared__ int32_t s_Wf[kMaxR];
+  __shared__ int32_t s_se[kMaxR * kMaxS];
+  __shared__ int32_t s_sq[kMaxR * kMaxS];
+  __shared__ int32_t s_cmax[kMaxJ], s_crep[kMaxJ], s_cstop[kMaxJ];
+  __shared__ int32_t s_best, s_A, s_iter_cap_hit;
+  __shared__ int32_t s_base[kMaxR + 1];
+
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int R = d.R, E = d.E, S = d.S, m = d.m;
+
+  for (int e = tid; e < E; e += nthr) {
+    int acc = 0;
+    for (int r = 0; r < R; ++r) acc += L.load[r * E + e];
+    Tot[e] = acc;
+    L.expert_total[e] = acc;
+  }
+  if (tid == 0) s_iter_cap_hit = 0;
+  __syncthreads();
+  if (tid < R) {
+    const int f = nat_first(tid, E, R), n = nat_count(tid, E, R);
+    int w = 0;
+    for (int i = 0; i < n; ++i) w += Tot[f + i];
+    s_W0[tid] = w;
+    L.W0[tid] = w;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int a = 0;
+    for (int q = lane; q < R; q += 32) a += s_W0[q];
+    a = __reduce_add_sync(kFull, a);
+    if (lane == 0) s_A = a;
+  }
+  __syncthreads();
+  const int A = s_A;
+
+  // ---- one greedy run per warp ----
+  const bool solver = warp < d.J;
+  const int j = warp;
+  const int64_t den = 200LL * R;
+  const int C = (int)(((int64_t)A * (200 + j) + den - 1) / den);
+  int Wr[kRW], used[kRW], se[kRW][SMAX], sq[kRW][SMAX];
+  int replicas = 0, stop = -1, maxW = 0;
+  if (solver) {
+    int32_t* Qn = Qn_all + j * E;
+    for (int e = lane; e < E; e += 32) Qn[e] = Tot[e];
+    unsigned stuck = 0, slotlim = 0;
+#pragma unroll
+    for (int k = 0; k < kRW; ++k) {
+      const int q = lane + 32 * k;
+      Wr[k] = q < R ? s_W0[q] : 0;
+      used[k] = 0;
+#pragma unroll
+      for (int t = 0; t < SMAX; ++t) { se[k][t] = -1; sq[k][t] = 0; }
+    }
+    __syncwarp();
+    const int iter_cap = 4 * (R * S + R + E) + 64;
+    for (int it = 0;; ++it) {
+      if (it >= iter_cap) { stop = EP_STOP_ITER_CAP; break; }
+      unsigned lm = 0;
+#pragma unroll
+      for (int k = 0; k < kRW; ++k)
+        if (lane + 32 * k < R && !((stuck >> k) & 1u)) lm = max(lm, (unsigned)Wr[k]);
+      const int vmax = (int)__reduce_max_sync(kFull, lm);
+      if (vmax <= C) break;
+      int p = -1;
+#pragma unroll
+      for (int k = 0; k < kRW; ++k) {
+        const unsigned b = __ballot_sync(
+            kFull, lane + 32 * k < R && !((stuck >> k) & 1u) && Wr[k] == vmax);
+        if (p < 0 && b) p = 32 * k + __ffs(b) - 1;
+      }
+      const int ex = vmax - C;
+      const int nf = nat_first(p, E, R), nc = nat_count(p, E, R);
+      const int myQ = lane < nc ? Qn[nf + lane] : 0;
+      bool tried = false, moved = false;
+      for (;;) {
+        const unsigned cq = (lane < nc && !tried && myQ >= m) ? (unsigned)myQ : 0u;
+        const unsigned qmax = __reduce_max_sync(kFull, cq);
+        if (qmax == 0) break;
+        const int li = __ffs(__ballot_sync(kFull, cq == qmax)) - 1;
+        const int e = nf + li;
+        // receivers: free slot, no instance of e, slack >= m
+        unsigned ls = 0;
+        bool ok[kRW];
+#pragma unroll
+        for (int k = 0; k < kRW; ++k) {
+          const int q = lane + 32 * k;
+          bool h = false;
+#pragma unroll
+          for (int t = 0; t < SMAX; ++t) h |= (se[k][t] == e);
+          ok[k] = q < R && q != p && used[k] < S && !h && C - Wr[k] >= m;
+          if (ok[k]) ls = max(ls, (unsigned)(C - Wr[k]));
+        }
+        const unsigned smax = __reduce_max_sync(kFull, ls);
+        if (smax == 0) {
+          if (lane == li) tried = true;
+          continue;
+        }
+        int rr = -1;
+#pragma unroll
+        for (int k = 0; k < kRW; ++k) {
+          const unsigned b = __ballot_sync(kFull, ok[k] && (unsigned)(C - Wr[k]) == smax);
+          if (rr < 0 && b) rr = 32 * k + __ffs(b) - 1;
+        }
+        const int x = min(min(max(ex, m), (int)smax), (int)qmax);
+#pragma unroll
+        for (int k = 0; k < kRW; ++k) {
+          const int q = lane + 32 * k;
+          if (q == p) Wr[k] -= x;
+          if (q == rr) {
+            Wr[k] += x;
+#pragma unroll
+            for (int t = 0; t < SMAX; ++t) {
+              const bool here = (t == used[k]);
+              se[k][t] = here ? e : se[k][t];
+              sq[k][t] = here ? x : sq[k][t];
+            }
+            used[k] += 1;
+          }
+        }
+        if (lane == li) Qn[e] = (int)qmax - x;
+        ++replicas;
+        moved = true;
+        break;
+      }
+      if (!moved) {
+        bool fr = false;
+#pragma unroll
+        for (int k = 0; k < kRW; ++k)
+          fr |= (lane + 32 * k < R && used[k] == S && C - Wr[k] >= m);
+        const bool full_receiver = __any_sync(kFull, fr);
+        const bool native_big = __any_sync(kFull, lane < nc && myQ >= m);
+#pragma unroll
+        for (int k = 0; k < kRW; ++k)
+          if (lane + 32 * k == p) {
+            stuck |= 1u << k;
+            if (full_receiver && native_big) slotlim |= 1u << k;
+          }
+      }
+      __syncwarp();
+    }
+    unsigned wm = 0;
+    bool sl = false;
+#pragma unroll
+    for (int k = 0; k < kRW; ++k)
+      if (lane + 32 * k < R) {
+        wm = max(wm, (unsigned)Wr[k]);
+        sl |= ((stuck >> k) & 1u) && ((slotlim >> k) & 1u) && Wr[k] > C;
+      }
+    maxW = (int)__reduce_max_sync(kFull, wm);
+    const bool any_sl = __any_sync(kFull, sl);
+    if (stop != EP_STOP_ITER_CAP)
+      stop = maxW <= C ? EP_STOP_BALANCED : (any_sl ? EP_STOP_SLOT_LIMITED : EP_STOP_QUOTA_LIMITED);
+    if (lane == 0) {
+      s_cmax[j] = maxW;
+      s_crep[j] = replicas;
+      s_cstop[j] = stop;
+      L.cand[j] = maxW;
+      L.cand[d.J + j] = replicas;
+      L.cand[2 * d.J + j] = stop;
+      if (stop == EP_STOP_ITER_CAP) atomicOr(&s_iter_cap_hit, 1);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {  // smallest (max load, replicas, j)
+    int b = 0;
+    for (int jj = 1; jj < d.J; ++jj)
+      if (s_cmax[jj] < s_cmax[b] || (s_cmax[jj] == s_cmax[b] && s_crep[jj] < s_crep[b])) b = jj;
+    s_best = b;
+  }
+  __syncthreads();
+  if (solver && j == s_best) {
+#pragma unroll
+    for (int k = 0; k < kRW; ++k) {
+      const int q = lane + 32 * k;
+      if (q < R) {
+        s_Wf[q] = Wr[k];
+        L.W[q] = Wr[k];
+#pragma unroll
+        for (int t = 0; t < SMAX; ++t)
+          if (t < S) { s_se[q * S + t] = se[k][t]; s_sq[q * S + t] = sq[k][t]; }
+      }
+    }
+    if (lane == 0) {
+      ep_layer_stats* st = L.stats;
+      st->cap_idx = j;
+      st->stop_reason = stop;
+      st->tight_stop_reason = s_cstop[0];
+      st->replicas = replicas;
+      st->cap = C;
+      st->assignments = A;
+      st->after_max = maxW;
+      if (s_iter_cap_hit) atomicOr(&st->status, EP_DEV_ITER_CAP);
+    }
+  }
+  __syncthreads();
+
+  // ---- emit the winner's instance table ----
+  const int G = d.G, Gmax = d.Gmax;
+  const int32_t* Qw = Qn_all + s_best * E;
+  for (int i = tid; i < R * G; i += nthr) {
+    const int q = i / G, col = i - (i / G) * G;
+    int ex = -1, qu = 0;
+    if (col < Gmax) {
+      if (col < nat_count(q, E, R)) { ex = nat_first(q, E, R) + col; qu = Qw[ex]; }
+    } else if (col < Gmax + S) {
+      ex = s_se[q * S + col - Gmax];
+      qu = s_sq[q * S + col - Gmax];
+    } else {
+      ex = E;  // the shared-expert column
+    }
+    L.inst_expert[i] = ex;
+    L.inst_quota[i] = qu;
+  }
+  for (int i = tid; i <= E; i += nthr) cnt_e[i] = 0;
+  __syncthreads();
+  if (tid < R) {  // rank-relative first row of every instance
+    int run = 0;
+    for (int col = 0; col < G; ++col) {
+      s.inst_rel[tid * G + col] = run;
+      int qu = 0;
+      if (col < Gmax) {
+        if (col < nat_count(tid, E, R)) qu = Qw[nat_first(tid, E, R) + col];
+      } else if (col < Gmax + S) {
+        qu = s_sq[tid * S + col - Gmax];
+      }
+      run += qu;
+    }
+  }
+  for (int i = tid; i < R * S; i += nthr)
+    if (s_se[i] >= 0) atomicAdd(&cnt_e[s_se[i]], 1);
+  if (warp == 0) {
+    // first row of each rank's block (routed rows only; a shared column moves it later)
+    int carry = 0;
+    for (int q0 = 0; q0 < R; q0 += 32) {
+      const int q = q0 + lane;
+      const int v = q < R ? s_Wf[q] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (q < R) s_base[q] = carry + incl - v;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) s_base[R] = carry;
+  }
+  __syncthreads();
+  if (!d.sh) {
+    for (int i = tid; i < R * G; i += nthr) L.inst_off[i] = s_base[i / G] + s.inst_rel[i];
+    if (tid == 0) L.inst_off[R * G] = s_base[R];
+    for (int q = tid; q <= R; q += nthr) L.rank_base[q] = s_base[q];
+    if (tid == 0) L.stats->rows = s_base[R];
+  } else {
+    // Waterfill waterline on the routed loads: H = ceil((sum W + N)/R),
+    // B = ceil(H * bonus / 1000), slack = max(H - W, 0).
+    const int64_t N = (int64_t)R * d.T;
+    const int64_t H = ((int64_t)A + N + R - 1) / R;
+    if (tid == 0) {
+      s.wf[0] = (int)H;
+      s.wf[1] = (int)((H * d.bonus + 999) / 1000);
+    }
+    for (int q = tid; q < R; q += nthr) s.slack[q] = (int)max(H - (int64_t)s_Wf[q], (int64_t)0);
+  }
+  if (tid == 0) {
+    int bm = 0;
+    for (int q = 0; q < R; ++q) bm = max(bm, s_W0[q]);
+    L.stats->before_max = bm;
+  }
+  // replica lists grouped by expert (CSR), instance order inside an expert
+  if (warp == 0) {
+    int carry = 0, ncarry = 0;
+    for (int e0 = 0; e0 <= E; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = e < E ? cnt_e[e] : 0;
+      const int f = v > 0 ? 1 : 0;
+      int incl = v, fincl = f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        const int z = __shfl_up_sync(kFull, fincl, o);
+        if (lane >= o) { incl += y; fincl += z; }
+      }
+      if (e <= E) L.rep_eptr[e] = carry + incl - v;
+      if (e < E && f) L.rep_experts[ncarry + fincl - 1] = e;
+      carry += __shfl_sync(kFull, incl, 31);
+      ncarry += __shfl_sync(kFull, fincl, 31);
+    }
+    if (lane == 0) L.rep_nexp[0] = ncarry;
+  }
+  __syncthreads();
+  for (int i = tid; i < R * S; i += nthr) {
+    const int e = s_se[i];
+    if (e < 0) continue;
+    int before = 0;
+    for (int i2 = 0; i2 < i; ++i2) before += (s_se[i2] == e);
+    L.rep_list[L.rep_eptr[e] + before] = i;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a3: local-first rerouting, one warp per expert.  Instances of e (native plus
+// replicas) in instance order; each source rank first uses the instance on its
+// own rank up to its quota; the residual demands, laid end to end in source
+// order, fill the residual quotas laid end to end in instance order.  The
+// output is, per (expert, source), the ordered segments (first ordinal,
+// destination rank, first row relative to that rank's block).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBuf L, Scratch s) {
+  __shared__ int32_t s_irank[kWarpsPerBlock][kMaxR];  // instance j: rank
+  __shared__ int32_t s_irel[kWarpsPerBlock][kMaxR];   // instance j: rank-relative first row
+  __shared__ int32_t s_iq[kWarpsPerBlock][kMaxR];     // instance j: quota, then residual
+  __shared__ int32_t s_ipq[kWarpsPerBlock][kMaxR];    // instance j: start of residual interval
+  __shared__ int32_t s_iloc[kWarpsPerBlock][kMaxR];   // instance j: local take
+  __shared__ int32_t s_jof[kWarpsPerBlock][kMaxR];    // rank -> instance j or -1
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * kWarpsPerBlock + warp;
+  if (e >= d.E) return;
+  const int R = d.R, E = d.E, G = d.G, S = d.S;
+  int32_t* irank = s_irank[warp];
+  int32_t* irel = s_irel[warp];
+  int32_t* iq = s_iq[warp];
+  int32_t* ipq = s_ipq[warp];
+  int32_t* iloc = s_iloc[warp];
+  int32_t* jof = s_jof[warp];
+
+  const int h = home_of(e, E, R);
+  const int hcol = e - nat_first(h, E, R);
+  const int p0 = L.rep_eptr[e], nrep = L.rep_eptr[e + 1] - p0;
+  const int ninst = nrep + 1;
+  // position of the native among the instances (replicas are in rank order)
+  int np = 0;
+  for (int j = lane; j < nrep; j += 32) np += (L.rep_list[p0 + j] / S) < h;
+  np = __reduce_add_sync(kFull, np);
+  for (int q = lane; q < R; q += 32) jof[q] = -1;
+  __syncwarp();
+  for (int j = lane; j < ninst; j += 32) {
+    int rank, col;
+    if (j == np) {
+      rank = h;
+      col = hcol;
+    } else {
+      const int slot = L.rep_list[p0 + (j < np ? j : j - 1)];
+      rank = slot / S;
+      col = d.Gmax + (slot - rank * S);
+    }
+    irank[j] = rank;
+    irel[j] = s.inst_rel[rank * G + col];
+    iq[j] = L.inst_quota[rank * G + col];
+    jof[rank] = j;
+  }
+  __syncwarp();
+  // local take and residual demand of every source rank (lane owns r = lane + 32k)
+  int Dr[kRW], locr[kRW];
+#pragma unroll
+  for (int k = 0; k < kRW; ++k) {
+    const int r = lane + 32 * k;
+    Dr[k] = 0;
+    locr[k] = 0;
+    if (r < R) {
+      const int l = L.load[r * E + e];
+      const int j = jof[r];
+      const int loc = j >= 0 ? min(l, iq[j]) : 0;
+      locr[k] = loc;
+      Dr[k] = l - loc;
+      if (j >= 0) iloc[j] = loc;
+    }
+  }
+  __syncwarp();
+  // residual quotas and their exclusive prefix in instance order
+  {
+    int carry = 0;
+    for (int j0 = 0; j0 < ninst; j0 += 32) {
+      const int j = j0 + lane;
+      const int v = j < ninst ? iq[j] - iloc[j] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (j < ninst) { iq[j] = v; ipq[j] = carry + incl - v; }
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+  }
+  __syncwarp();
+  // exclusive prefix of residual demand in source order
+  int PD[kRW];
+  {
+    int carry = 0;
+#pragma unroll
+    for (int k = 0; k < kRW; ++k) {
+      int incl = Dr[k];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      PD[k] = carry + incl - Dr[k];
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+  }
+  // first instance whose residual interval ends after PD (binary search)
+  auto first_after = [&](int x) {
+    int lo = 0, hi = ninst;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (ipq[mid] + iq[mid] > x) hi = mid; else lo = mid + 1;
+    }
+    return lo;
+  };
+  // pass 1: segment count per source, prefix in source order
+  int cnt[kRW], j0r[kRW];
+#pragma unroll
+  for (int k = 0; k < kRW; ++k) {
+    cnt[k] = 0;
+    j0r[k] = 0;
+    const int r = lane + 32 * k;
+    if (r < R) {
+      cnt[k] = locr[k] > 0 ? 1 : 0;
+      if (Dr[k] > 0) {
+        const int end = PD[k] + Dr[k];
+        int j = first_after(PD[k]);
+        j0r[k] = j;
+        for (; j < ninst && ipq[j] < end; ++j) cnt[k] += iq[j] > 0;
+      }
+    }
+  }
+  int segbase[kRW];
+  {
+    int carry = 0;
+#pragma unroll
+    for (int k = 0; k < kRW; ++k) {
+      int incl = cnt[k];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      segbase[k] = carry + incl - cnt[k];
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) s.seg_ptr[e * (R + 1) + R] = carry;
+  }
+  // pass 2: write the segments
+  int32_t* sord = s.seg_ord + (int64_t)e * 3 * R;
+  int32_t* srank = s.seg_rank + (int64_t)e * 3 * R;
+  int32_t* srel = s.seg_rel + (int64_t)e * 3 * R;
+#pragma unroll
+  for (int k = 0; k < kRW; ++k) {
+    const int r = lane + 32 * k;
+    if (r >= R) continue;
+    s.seg_ptr[e * (R + 1) + r] = segbase[k];
+    int w = segbase[k];
+    if (locr[k] > 0) {
+      const int j = jof[r];
+      const int before = min(max(PD[k] - ipq[j], 0), iq[j]);  // remote rows of earlier sources
+      sord[w] = 0;
+      srank[w] = r;
+      srel[w] = irel[j] + before;
+      ++w;
+    }
+    if (Dr[k] > 0) {
+      const int end = PD[k] + Dr[k];
+      for (int j = j0r[k]; j < ninst && ipq[j] < end; ++j) {
+        if (iq[j] <= 0) continue;
+        const int lo = max(PD[k], ipq[j]);
+        const int c = irank[j];
+        sord[w] = locr[k] + (lo - PD[k]);
+        srank[w] = c;
+        srel[w] = irel[j] + (c < r ? iloc[j] : 0) + (lo - ipq[j]);
+        ++w;
+      }
+    }
+  }
+}
+
+// Set / clear bit q of a 4-word rank mask without a dynamic word index.
+__device__ __forceinline__ void mask_set(unsigned (&mask)[kRW], int q) {
+  const unsigned bit = 1u << (q & 31);
+#pragma unroll
+  for (int w = 0; w < kRW; ++w) mask[w] |= (q >> 5) == w ? bit : 0u;
+}
+__device__ __forceinline__ void mask_clear(unsigned (&mask)[kRW], int q) {
+  const unsigned bit = 1u << (q & 31);
+#pragma unroll
+  for (int w = 0; w < kRW; ++w) mask[w] &= (q >> 5) == w ? ~bit : ~0u;
+}
+
+// ---------------------------------------------------------------------------
+// a5 device side: the Waterfill pick of one token.  cand mask holds the ranks
+// the token visits; the own rank r comes first, the others ascending.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int wf_pick(int r, int64_t token, const unsigned (&mask)[kRW],
+                                       const int32_t* slack, const int32_t* W, int B,
+                                       uint64_t seed) {
+  int64_t sumS = slack[r];
+#pragma unroll
+  for (int w = 0; w < kRW; ++w) {
+    unsigned b = mask[w];
+    while (b) {
+      const int c = 32 * w + __ffs(b) - 1;
+      b &= b - 1;
+      sumS += slack[c];
+    }
+  }
+  if (sumS > 0) {
+    const uint64_t h = splitmix64(seed + (uint64_t)token);
+    const uint64_t u = ((h >> 32) * (uint64_t)(sumS + B)) >> 32;
+    int64_t acc = (int64_t)slack[r] + B;
+    if ((uint64_t)acc > u) return r;
+    int last = r;
+#pragma unroll
+    for (int w = 0; w < kRW; ++w) {
+      unsigned b = mask[w];
+      while (b) {
+        const int c = 32 * w + __ffs(b) - 1;
+        b &= b - 1;
+        acc += slack[c];
+        last = c;
+        if ((uint64_t)acc > u) return c;
+      }
+    }
+    return last;
+  }
+  int lo = r;
+#pragma unroll
+  for (int w = 0; w < kRW; ++w) {
+    unsigned b = mask[w];
+    while (b) {
+      const int c = 32 * w + __ffs(b) - 1;
+      b &= b - 1;
+      if (W[c] < W[lo] || (W[c] == W[lo] && c < lo)) lo = c;
+    }
+  }
+  return W[r] <= W[lo] + B ? r : lo;
+}
+
+// ---------------------------------------------------------------------------
+// a4 (+a5): token assignment.  One warp per sub-chunk.  The stable ordinal of
+// (t, k) among its source rank's assignments of expert e = exclusive base of
+// the sub-chunk + running count in the warp + rank inside the 32-lane group;
+// the ordinal selects the (source, expert) segment and thus the row.
+// PASS 0: rows, no shared expert.  PASS 1: Waterfill picks, counted per
+// (destination rank, sub-chunk).  PASS 2: rows and shared-slot rows.
+// ---------------------------------------------------------------------------
+template <int PASS>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
+  extern __shared__ int32_t sm[];
+  __shared__ int32_t s_rb[kMaxR + 1];
+  __shared__ int32_t s_slack[kMaxR];
+  __shared__ int32_t s_W[kMaxR];
+  __shared__ int32_t s_sbase[kMaxR];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int R = d.R, E = d.E, K = d.K;
+  for (int q = threadIdx.x; q <= R; q += blockDim.x) {
+    if (PASS != 1) s_rb[q] = L.rank_base[q];
+    if (PASS > 0 && q < R) {
+      s_slack[q] = s.slack[q];
+      s_W[q] = L.W[q];
+      if (PASS == 2) s_sbase[q] = s.sbase[q];
+    }
+  }
+  __syncthreads();
+  const int gw = blockIdx.x * kWarpsPerBlock + warp;
+  if (gw >= R * d.nsub) return;
+  // per-warp shared: run[E] | wrun[R] | dr[kSubT*K] (uint8)
+  const int per_warp = E + (PASS > 0 ? R + (kSubT * K + 3) / 4 : 0);
+  int32_t* run = sm + warp * per_warp;
+  int32_t* wrun = run + E;
+  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);
+  const int r = gw / d.nsub, sub = gw - (gw / d.nsub) * d.nsub;
+  const int32_t* base = s.sub_cnt + (int64_t)gw * E;
+  for (int e = lane; e < E; e += 32) run[e] = base[e];
+  __syncwarp();
+  const int t0 = sub * kSubT, t1 = min(d.T, t0 + kSubT);
+  const int a0 = t0 * K, a1 = t1 * K;
+  const int64_t rbase = (int64_t)r * d.T * K;
+  const int32_t* seg_ptr = s.seg_ptr;
+  for (int a = a0; a < a1; a += 32) {
+    const int idx = a + lane;
+    int e = -1;
+    if (idx < a1) {
+      e = __ldg(ids + rbase + idx);
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(kFull, e);
+    const int rk = __popc(peers & lanemask_lt());
+    const int o = e >= 0 ? run[e] + rk : 0;
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) run[e] = o + __popc(peers);  // leader: rk = 0
+    __syncwarp();
+    if (idx < a1) {
+      int row = -1, rank = kNoRank;
+      if (e >= 0) {
+        const int sp = e * (R + 1) + r;
+        const int s0 = seg_ptr[sp], s1 = seg_ptr[sp + 1];
+        const int64_t sb = (int64_t)e * 3 * R;
+        int si = s1 - 1;
+        while (si > s0 && s.seg_ord[sb + si] > o) --si;
+        const int rk = (s1 > s0 && s0 >= 0 && s1 <= 3 * R) ? s.seg_rank[sb + si] : -1;
+        if (rk >= 0 && rk < R) {
+          rank = rk;
+          const int rel = s.seg_rel[sb + si] + (o - s.seg_ord[sb + si]);
+          if (PASS != 1) row = s_rb[rank] + rel;
+        } else {
+          atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
+        }
+      }
+      if (PASS != 1) L.dst_row[rbase + idx] = row;
+      if (PASS > 0) dr[idx - a0] = (uint8_t)rank;
+    }
+  }
+  if (PASS > 0) {
+    for (int q = lane; q < R; q += 32)
+      wrun[q] = PASS == 1 ? 0 : s.wsub_cnt[(int64_t)q * R * d.nsub + gw];
+    __syncwarp();
+    const int B = s.wf[1];
+    for (int t = t0; t < t1; t += 32) {
+      const int tt = t + lane;
+      int c = -1;
+      if (tt < t1) {
+        unsigned mask[kRW] = {0u, 0u, 0u, 0u};
+        for (int k = 0; k < K; ++k) {
+          const int q = dr[(tt - t0) * K + k];
+          if (q != kNoRank) mask_set(mask, q);
+        }
+        mask_clear(mask, r);
+        c = wf_pick(r, (int64_t)r * d.T + tt, mask, s_slack, s_W, B, d.seed);
+      }
+      const unsigned peers = __match_any_sync(kFull, c);
+      const int rk = __popc(peers & lanemask_lt());
+      const int o = c >= 0 ? wrun[c] + rk : 0;
+      __syncwarp();
+      if (c >= 0 && lane == __ffs(peers) - 1) wrun[c] = o + __popc(peers);
+      __syncwarp();
+      if (PASS == 2 && tt < t1) {
+        L.shared_rank[(int64_t)r * d.T + tt] = c;
+        L.shared_row[(int64_t)r * d.T + tt] = s_sbase[c] + o;
+      }
+    }
+    if (PASS == 1) {
+      __syncwarp();
+      for (int q = lane; q < R; q += 32) s.wsub_cnt[(int64_t)q * R * d.nsub + gw] = wrun[q];
+    }
+  }
+}
+
+// Shared-slot layout: for each destination rank c, exclusive scan of its pick
+// counts over (source rank, sub-chunk) — rows ordered by (source rank, token) —
+// then every rank's block = routed rows followed by its shared column.
+__global__ void __launch_bounds__(1024) k_shared_scan(Dims d, LayerBuf L, Scratch s) {
+  __shared__ int32_t s_tot[kMaxR];
+  __shared__ int32_t s_base[kMaxR + 1];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const int R = d.R, G = d.G;
+  const int n = R * d.nsub;
+  for (int c = warp; c < R; c += nw) {
+    int32_t* col = s.wsub_cnt + (int64_t)c * n;
+    int carry = 0;
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      const int v = i < n ? col[i] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (i < n) col[i] = carry + incl - v;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) s_tot[c] = carry;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int q0 = 0; q0 < R; q0 += 32) {
+      const int q = q0 + lane;
+      const int v = q < R ? L.W[q] + s_tot[q] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (q < R) s_base[q] = carry + incl - v;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    if (lane == 0) s_base[R] = carry;
+  }
+  __syncthreads();
+  const int scol = d.Gmax + d.S;
+  for (int i = threadIdx.x; i < R * G; i += blockDim.x) {
+    const int q = i / G, col = i - (i / G) * G;
+    if (col == scol) {
+      L.inst_quota[i] = s_tot[q];
+      L.inst_off[i] = s_base[q] + L.W[q];
+    } else {
+      L.inst_off[i] = s_base[q] + s.inst_rel[i];
+    }
+  }
+  for (int q = threadIdx.x; q <= R; q += blockDim.x) {
+    L.rank_base[q] = s_base[q];
+    if (q < R) s.sbase[q] = s_base[q] + L.W[q];
+  }
+  if (threadIdx.x == 0) {
+    L.inst_off[R * G] = s_base[R];
+    L.stats->rows = s_base[R];
+  }
+}
+
+// Standalone Waterfill: one thread per token; the waterline is recomputed per
+// block from the loads (R <= 128 values).
+__global__ void __launch_bounds__(256)
+k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
+            const int32_t* __restrict__ dst_rank, uint64_t seed, int bonus,
+            int32_t* __restrict__ pick, int32_t* __restrict__ count) {
+  __shared__ int32_t s_load[kMaxR], s_slack[kMaxR];
+  __shared__ int64_t s_sum;
+  if (threadIdx.x == 0) s_sum = 0;
+  __syncthreads();
+  for (int q = threadIdx.x; q < R; q += blockDim.x) {
+    s_load[q] = load[q];
+    atomicAdd(reinterpret_cast<unsigned long long*>(&s_sum), (unsigned long long)load[q]);
+  }
+  __syncthreads();
+  const int64_t N = (int64_t)R * T;
+  const int64_t H = (s_sum + N + R - 1) / R;
+  const int B = (int)((H * bonus + 999) / 1000);
+  for (int q = threadIdx.x; q < R; q += blockDim.x)
+    s_slack[q] = (int)max(H - (int64_t)s_load[q], (int64_t)0);
+  __syncthreads();
+  const int64_t tok = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tok >= N) return;
+  const int r = (int)(tok / T);
+  unsigned mask[kRW] = {0u, 0u, 0u, 0u};
+  for (int k = 0; k < K; ++k) {
+    const int q = dst_rank[tok * K + k];
+    if (q >= 0 && q < R) mask_set(mask, q);
+  }
+  mask_clear(mask, r);
+  const int c = wf_pick(r, tok, mask, s_slack, s_load, B, seed);
+  pick[tok] = c;
+  atomicAdd(&count[c], 1);
+}
+
+template <int SMAX>
+cudaError_t set_solve_attr(size_t smem) {
+  return cudaFuncSetAttribute(k_solve<SMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+size_t solve_smem(const Dims& d) { return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + d.E + 1); }
+size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
+size_t assign_smem(const Dims& d, int pass) {
+  const int per_warp = d.E + (pass > 0 ? d.R + (kSubT * d.K + 3) / 4 : 0);
+  return sizeof(int32_t) * (size_t)kWarpsPerBlock * per_warp;
+}
+
+}  // namespace
+
+cudaError_t set_plan_attributes(const Dims& d) {
+  cudaError_t e = cudaSuccess;
+  const size_t ss = solve_smem(d);
+  if (d.S <= 1) e = set_solve_attr<1>(ss);
+  else if (d.S <= 2) e = set_solve_attr<2>(ss);
+  else if (d.S <= 4) e = set_solve_attr<4>(ss);
+  else e = set_solve_attr<8>(ss);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem(d));
+  if (e != cudaSuccess) return e;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int sm = (int)assign_smem(d, pass);
+    if (pass == 0) e = cudaFuncSetAttribute(k_assign<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (pass == 1) e = cudaFuncSetAttribute(k_assign<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (pass == 2) e = cudaFuncSetAttribute(k_assign<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, const int32_t* ids,
+                           cudaStream_t st) {
+  cudaError_t err = cudaMemsetAsync(L.stats, 0, sizeof(ep_layer_stats), st);
+  if (err != cudaSuccess) return err;
+  const int nwarps = d.R * d.nsub;
+  const int nblk = (nwarps + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  if (nblk > 0) k_hist<<<nblk, kWarpsPerBlock * 32, hist_smem(d), st>>>(ids, d, s, L.stats);
+  k_scan<<<(d.R * d.E + 255) / 256, 256, 0, st>>>(d, s, L);
+  const size_t ss = solve_smem(d);
+  const int sthreads = kMaxJ * 32;
+  if (d.S <= 1) k_solve<1><<<1, sthreads, ss, st>>>(d, L, s);
+  else if (d.S <= 2) k_solve<2><<<1, sthreads, ss, st>>>(d, L, s);
+  else if (d.S <= 4) k_solve<4><<<1, sthreads, ss, st>>>(d, L, s);
+  else k_solve<8><<<1, sthreads, ss, st>>>(d, L, s);
+  k_reroute<<<(d.E + kWarpsPerBlock - 1) / kWarpsPerBlock, kWarpsPerBlock * 32, 0, st>>>(d, L, s);
+  if (!d.sh) {
+    if (nblk > 0) k_assign<0><<<nblk, kWarpsPerBlock * 32, assign_smem(d, 0), st>>>(ids, d, L, s);
+  } else {
+    if (nblk > 0) k_assign<1><<<nblk, kWarpsPerBlock * 32, assign_smem(d, 1), st>>>(ids, d, L, s);
+    k_shared_scan<<<1, 1024, 0, st>>>(d, L, s);
+    if (nblk > 0) k_assign<2><<<nblk, kWarpsPerBlock * 32, assign_smem(d, 2), st>>>(ids, d, L, s);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_waterfill(int R, int T, int K, const int32_t* load, const int32_t* dst_rank,
+                             uint64_t seed, int bonus, int32_t* pick, int32_t* count,
+                             cudaStream_t st) {
+  cudaError_t err = cudaMemsetAsync(count, 0, sizeof(int32_t) * (size_t)R, st);
+  if (err != cudaSuccess) return err;
+  const int64_t N = (int64_t)R * T;
+  if (N > 0)
+    k_waterfill<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(R, T, K, load, dst_rank, seed, bonus,
+                                                             pick, count);
+  return cudaGetLastError();
+}
+
+}  // namespace ep

@@ -210,6 +210,16 @@ def permute(p: Plan, hidden: np.ndarray) -> np.ndarray:
     return out
 
 
+def permute_range(p: Plan, hidden_rows: np.ndarray, n0: int, out: np.ndarray) -> None:
+    """Dispatch tokens [n0, n0 + len(hidden_rows)) of the layer into `out` (all rows)."""
+    hidden_rows = np.ascontiguousarray(hidden_rows)
+    n = hidden_rows.shape[0]
+    assert out.flags.c_contiguous and out.strides[0] == hidden_rows.strides[0]
+    dst = np.ascontiguousarray(p.dst_row.reshape(-1, p.K)[n0:n0 + n])
+    srow = None if p.shared_row is None else np.ascontiguousarray(p.shared_row.reshape(-1)[n0:n0 + n])
+    _load().orc_permute(n, p.K, hidden_rows.strides[0], _p(hidden_rows), _p(dst), _p(srow), _p(out))
+
+
 def stage(p: Plan, native_w: np.ndarray, slots: np.ndarray) -> None:
     """slots[q][s] = native_w[expert of slot (q, s)] for every filled slot (in place)."""
     native_w = np.ascontiguousarray(native_w)

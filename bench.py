@@ -134,6 +134,24 @@ def _dist_init():
     return world, rank, local
 
 
+def _workload(args):
+    """The named workload; --tokens-per-rank / --ffn shrink it for profiler captures."""
+    from workloads import get_config
+
+    w = get_config(args.workload)
+    if w.layers > 1:
+        w = w.replace(layers=1)
+    over = {}
+    if args.tokens_per_rank is not None:
+        over["T"] = args.tokens_per_rank
+    if args.ffn is not None:
+        over["ffn"] = args.ffn
+    if over:
+        tag = ",".join(f"{k}={v}" for k, v in over.items())
+        w = w.replace(name=f"{w.name}[{tag}]", **over)
+    return w
+
+
 def run_gpu(args):
     import datetime
 
@@ -151,9 +169,7 @@ def run_gpu(args):
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    w = get_config(args.workload)
-    if w.layers > 1:
-        w = w.replace(layers=1)
+    w = _workload(args)
     dev = torch.device("cuda", local)
     ids_np = topk_ids(w)
     ids = torch.from_numpy(ids_np).to(dev)
@@ -381,11 +397,7 @@ def run_reference(args):
     world, rank, _ = _dist_init()
     if rank != 0:
         return None
-    from workloads import get_config
-
-    w = get_config(args.workload)
-    if w.layers > 1:
-        w = w.replace(layers=1)
+    w = _workload(args)
     for _ in range(max(0, args.warmup)):
         cpu_baseline(w, steps=1)
     steps = max(1, args.steps)
@@ -415,6 +427,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens-per-rank", type=int, default=None,
+                    help="override T (small cases for profiler captures)")
+    ap.add_argument("--ffn", type=int, default=None, help="override the expert FFN width")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "cuda":
         ap.error("--warmup must be at least 3")

@@ -10,8 +10,8 @@
 #include "ep_internal.cuh"
 
 namespace ep {
-cudaError_t set_plan_attributes(const Dims& d);
-cudaError_t set_copy_attributes(const Dims& d);
+cudaError_t set_plan_attributes(int max_smem);
+cudaError_t set_copy_attributes(int max_smem);
 }  // namespace ep
 
 namespace {
@@ -227,8 +227,11 @@ ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t works
   if (cudaGetDevice(&dev) != cudaSuccess) return EP_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return EP_ERR_CUDA;
-  if (ep::set_plan_attributes(d) != cudaSuccess) return EP_ERR_CUDA;
-  if (ep::set_copy_attributes(d) != cudaSuccess) return EP_ERR_CUDA;
+  int max_smem = 0;
+  if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return EP_ERR_CUDA;
+  if (ep::set_plan_attributes(max_smem) != cudaSuccess) return EP_ERR_CUDA;
+  if (ep::set_copy_attributes(max_smem) != cudaSuccess) return EP_ERR_CUDA;
   ep_plan* p = new (std::nothrow) ep_plan;
   if (!p) return EP_ERR_INVALID_ARGUMENT;
   p->planned = new (std::nothrow) unsigned char[cfg->num_layers];

@@ -350,13 +350,11 @@ int permute_ctas_per_sm(uint32_t row_bytes) {
 
 }  // namespace
 
-cudaError_t set_copy_attributes(const Dims& d) {
-  const size_t psmem = 128 + (size_t)kStages * (size_t)d.hidden * 2;
-  cudaError_t e =
-      cudaFuncSetAttribute(k_permute, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+cudaError_t set_copy_attributes(int max_smem) {
+  const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e = cudaFuncSetAttribute(k_permute, a, max_smem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_stage, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              128 + kStages * kStageTile);
+  return cudaFuncSetAttribute(k_stage, a, max_smem);
 }
 
 cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden, void* out,

@@ -93,6 +93,5 @@ cudaError_t launch_reduce(const Dims& d, const LayerBuf& L, void* slot_grads, in
 cudaError_t launch_waterfill(int R, int T, int K, const int32_t* load, const int32_t* dst_rank,
                              uint64_t seed, int bonus, int32_t* pick, int32_t* count,
                              cudaStream_t st);
-cudaError_t set_kernel_attributes(const Dims& d);
 
 }  // namespace ep

@@ -871,8 +871,8 @@ k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
 }
 
 template <int SMAX>
-cudaError_t set_solve_attr(size_t smem) {
-  return cudaFuncSetAttribute(k_solve<SMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t set_solve_attr(int smem) {
+  return cudaFuncSetAttribute(k_solve<SMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
 }
 
 size_t solve_smem(const Dims& d) { return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + d.E + 1); }
@@ -884,24 +884,19 @@ size_t assign_smem(const Dims& d, int pass) {
 
 }  // namespace
 
-cudaError_t set_plan_attributes(const Dims& d) {
-  cudaError_t e = cudaSuccess;
-  const size_t ss = solve_smem(d);
-  if (d.S <= 1) e = set_solve_attr<1>(ss);
-  else if (d.S <= 2) e = set_solve_attr<2>(ss);
-  else if (d.S <= 4) e = set_solve_attr<4>(ss);
-  else e = set_solve_attr<8>(ss);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_smem(d));
-  if (e != cudaSuccess) return e;
-  for (int pass = 0; pass < 3; ++pass) {
-    const int sm = (int)assign_smem(d, pass);
-    if (pass == 0) e = cudaFuncSetAttribute(k_assign<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    if (pass == 1) e = cudaFuncSetAttribute(k_assign<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    if (pass == 2) e = cudaFuncSetAttribute(k_assign<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+// Allow every kernel the device's opt-in shared-memory maximum once, so that
+// plans of any shape can coexist (each launch still requests only its own size).
+cudaError_t set_plan_attributes(int max_smem) {
+  cudaError_t e;
+  if ((e = set_solve_attr<1>(max_smem)) != cudaSuccess) return e;
+  if ((e = set_solve_attr<2>(max_smem)) != cudaSuccess) return e;
+  if ((e = set_solve_attr<4>(max_smem)) != cudaSuccess) return e;
+  if ((e = set_solve_attr<8>(max_smem)) != cudaSuccess) return e;
+  const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  if ((e = cudaFuncSetAttribute(k_hist, a, max_smem)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(k_assign<0>, a, max_smem)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(k_assign<1>, a, max_smem)) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_assign<2>, a, max_smem);
 }
 
 cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, const int32_t* ids,

@@ -351,10 +351,9 @@ int permute_ctas_per_sm(uint32_t row_bytes) {
 }  // namespace
 
 cudaError_t set_copy_attributes(int max_smem) {
-  const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
-  cudaError_t e = cudaFuncSetAttribute(k_permute, a, max_smem);
+  cudaError_t e = allow_max_dynamic_smem(k_permute, max_smem);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_stage, a, max_smem);
+  return allow_max_dynamic_smem(k_stage, max_smem);
 }
 
 cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden, void* out,

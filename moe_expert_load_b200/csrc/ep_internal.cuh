@@ -80,6 +80,18 @@ __host__ __device__ __forceinline__ int home_of(int e, int E, int R) {
   return e < big ? e / (base + 1) : rem + (e - big) / base;
 }
 
+// Let kernel f request up to the device's opt-in shared memory per block:
+// static + dynamic shared memory may not exceed it, so the dynamic allowance is
+// the opt-in maximum minus f's static shared memory.
+template <typename F>
+inline cudaError_t allow_max_dynamic_smem(F* f, int max_smem) {
+  cudaFuncAttributes a;
+  cudaError_t e = cudaFuncGetAttributes(&a, f);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              max_smem - (int)a.sharedSizeBytes);
+}
+
 // ---- launchers (defined in the .cu files) ----------------------------------
 cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s,
                            const int32_t* ids, cudaStream_t st);

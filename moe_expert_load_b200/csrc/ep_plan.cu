@@ -870,11 +870,6 @@ k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
   atomicAdd(&count[c], 1);
 }
 
-template <int SMAX>
-cudaError_t set_solve_attr(int smem) {
-  return cudaFuncSetAttribute(k_solve<SMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-}
-
 size_t solve_smem(const Dims& d) { return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + d.E + 1); }
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
@@ -888,15 +883,14 @@ size_t assign_smem(const Dims& d, int pass) {
 // plans of any shape can coexist (each launch still requests only its own size).
 cudaError_t set_plan_attributes(int max_smem) {
   cudaError_t e;
-  if ((e = set_solve_attr<1>(max_smem)) != cudaSuccess) return e;
-  if ((e = set_solve_attr<2>(max_smem)) != cudaSuccess) return e;
-  if ((e = set_solve_attr<4>(max_smem)) != cudaSuccess) return e;
-  if ((e = set_solve_attr<8>(max_smem)) != cudaSuccess) return e;
-  const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
-  if ((e = cudaFuncSetAttribute(k_hist, a, max_smem)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(k_assign<0>, a, max_smem)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(k_assign<1>, a, max_smem)) != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_assign<2>, a, max_smem);
+  if ((e = allow_max_dynamic_smem(k_solve<1>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_solve<2>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_solve<4>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_solve<8>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_hist, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_assign<0>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_assign<1>, max_smem)) != cudaSuccess) return e;
+  return allow_max_dynamic_smem(k_assign<2>, max_smem);
 }
 
 cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, const int32_t* ids,

@@ -250,3 +250,20 @@ def test_errors_are_status_codes():
     plan.balance_layer(0, ids)
     with pytest.raises(EpError):
         plan.dispatch_layout(0, _hidden(w), rank_begin=3, rank_end=2)
+
+
+def test_plans_of_different_shapes_coexist():
+    # a plan with 14 KiB rows created before a plan with 512 B rows must still
+    # launch its dispatch (per-kernel shared-memory limits are plan independent)
+    wa = get_config("dsv3").replace(T=300)
+    ida = topk_ids(get_config("dsv3"))[:, :300].copy()
+    pa = gpu_plan(wa, ida)
+    wb = get_config("tiny")
+    pb = gpu_plan(wb, topk_ids(wb))
+    ha = _hidden(wa)
+    out = pa.dispatch_layout(0, ha)
+    pb.dispatch_layout(0, _hidden(wb))
+    torch.cuda.synchronize()
+    dst = pa.view(0)["dst_row"].reshape(wa.N, wa.K).long()
+    assert torch.equal(out[dst[:, 0]].view(torch.int16), ha.view(torch.int16))
+    assert pa.read_layer_stats(0)["status"] == 0 and pb.read_layer_stats(0)["status"] == 0

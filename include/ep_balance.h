@@ -230,6 +230,30 @@ EP_API ep_status_t ep_waterfill(int32_t R, int32_t T, int32_t K, const int32_t* 
                          const int32_t* d_dst_rank, uint64_t seed, int32_t bonus_permille,
                          int32_t* d_pick, int32_t* d_count, void* stream);
 
+/*
+ * Load matrix without allocation.  The pages have no counterpart: this exists
+ * for callers that cannot allocate device memory on this path (engines that
+ * reserve nearly all device memory up front, embedded callers without an
+ * allocator, loops where an allocation would synchronise the device).
+ * Computes d_load[r][e] = number of (t, k) with d_topk_ids[r][t][k] == e — the
+ * same values as ep_layer_view.load after ep_balance_layer — from d_topk_ids
+ * [R][T][K] int32 into d_load [R][E] int32 (both caller-owned device memory).
+ * d_status (device int32, may be NULL) is set to EP_DEV_BAD_ID if an id was
+ * outside [0, E), else 0; such ids are not counted.
+ * It calls no allocator: its only scratch, R*ceil(T/128)*E int32 sub-chunk
+ * counts, lives in a fixed device array of EP_LOAD_STATIC_MAX_SCRATCH int32
+ * (4 MiB) that every GPU loading the library holds until the process exits;
+ * larger shapes return EP_ERR_UNSUPPORTED.  The first call on each device looks
+ * up the array's address (cudaGetSymbolAddress) — make that first call before
+ * any stream capture.  All calls on a device share the array; calls that
+ * overlap on the GPU race and must be serialised by the caller.  Limits: R >= 1,
+ * 1 <= E <= 1024, 1 <= K <= 16, T >= 0, R*T*K < 2^31.  Asynchronous on `stream`.
+ */
+#define EP_LOAD_STATIC_MAX_SCRATCH (1 << 20)
+EP_API ep_status_t ep_load_matrix_static(int32_t R, int32_t E, int32_t K, int32_t T,
+                                         const int32_t* d_topk_ids, int32_t* d_load,
+                                         int32_t* d_status, void* stream);
+
 EP_API const char* ep_status_string(ep_status_t status);
 EP_API int32_t ep_abi_version(void);
 

@@ -27,6 +27,7 @@ EXPORTS = (
     "ep_plan_workspace_bytes", "ep_plan_create", "ep_plan_destroy", "ep_balance_layer",
     "ep_layer_view_get", "ep_read_layer_stats", "ep_dispatch_layout", "ep_stage_replicas",
     "ep_reduce_replica_grads", "ep_waterfill", "ep_status_string", "ep_abi_version",
+    "ep_load_matrix_static",
 )
 
 

@@ -152,6 +152,43 @@ def _workload(args):
     return w
 
 
+def _events(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def _timed(torch, fn, iters, stream, flush=None, skip=1):
+    """Device time (ms) of fn per call, CUDA events on `stream`; optional L2
+    flush (a write larger than L2) before each call."""
+    out = []
+    for k in range(iters + skip):
+        if flush is not None:
+            flush.fill_(k & 0xFF)
+        a, b = _events(torch)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        if k >= skip:
+            out.append(a.elapsed_time(b))
+    return out
+
+
+def _median(xs):
+    xs = sorted(xs)
+    return xs[len(xs) // 2]
+
+
+def _balance_launches(w):
+    return 3 + (3 if w.shared_expert else 1)  # hist, solve, reroute + assign pass(es)
+
+
+def _ratio(st, R):
+    A = max(1, int(st["assignments"]))
+    return {"before": st["before_max"] * R / A, "after": st["after_max"] * R / A,
+            "stop_reason": st["stop_reason"], "tight_stop_reason": st["tight_stop_reason"],
+            "replicas": st["replicas"], "cap_idx": st["cap_idx"]}
+
+
 def run_gpu(args):
     import datetime
 
@@ -159,7 +196,7 @@ def run_gpu(args):
     import torch
 
     from moe_expert_load_b200 import Plan, config_from_workload
-    from workloads import get_config, topk_ids
+    from workloads import topk_ids
 
     world, rank, local = _dist_init()
     torch.cuda.set_device(local)
@@ -173,17 +210,22 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     ids_np = topk_ids(w)
     ids = torch.from_numpy(ids_np).to(dev)
+    if args.plan_only:
+        return run_plan_only(args, w, ids, dev)
     g = torch.Generator(device=dev)
     g.manual_seed(1000 + rank)
     hidden = torch.randn((w.N, w.hidden), generator=g, device=dev).to(torch.bfloat16)
     native_w = torch.randn((w.E, w.expert_elems), generator=g, device=dev).to(torch.bfloat16)
     slots = torch.zeros((w.R, w.S, w.expert_elems), dtype=torch.bfloat16, device=dev)
+    slot_grads = (torch.randn((w.R, w.S, w.expert_elems), generator=g, device=dev) * 1e-2).to(torch.bfloat16)
+    native_grads = torch.zeros((w.E, w.expert_elems), dtype=torch.float32, device=dev)
     rows_cap = w.A + (w.N if w.shared_expert else 0)
     out = torch.empty((rows_cap, w.hidden), dtype=torch.bfloat16, device=dev)
     plan = Plan(config_from_workload(w, num_layers=1), device=dev)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
+        # forward: balance, stage replicas, dispatch
         plan.balance_layer(0, ids)
         plan.stage_replicas(0, native_w, slots)
         if ev is not None:
@@ -191,6 +233,9 @@ def run_gpu(args):
         plan.dispatch_layout(0, hidden, out=out)
         if ev is not None:
             ev[1].record(stream)
+        # backward: re-stage from the cached plan, reduce replica gradients
+        plan.stage_replicas(0, native_w, slots)
+        plan.reduce_replica_grads(0, slot_grads, native_grads)
 
     def barrier():
         if dist is not None:
@@ -200,13 +245,11 @@ def run_gpu(args):
     for _ in range(args.warmup):
         step()
     stats = plan.read_layer_stats(0)
-    launches_per_step = (4 + (3 if w.shared_expert else 1)) + 1 + 1  # balance + stage + dispatch
+    launches_per_step = _balance_launches(w) + 4  # + stage, dispatch, re-stage, reduce
 
     # ---- timed region: K whole steps --------------------------------------
-    perm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
+    perm_ev = [_events(torch) for _ in range(args.steps)]
+    t0, t1 = _events(torch)
     barrier()
     with ClockSampler(local) as clk:
         t0.record(stream)
@@ -224,39 +267,20 @@ def run_gpu(args):
     perm_ms = [a.elapsed_time(b) for a, b in perm_ev]
     perm_avg_ms = sum(perm_ms) / len(perm_ms)
 
-    # ---- plan latency alone, with L2 flushed before every call -------------
+    # ---- each piece alone, L2 flushed before every call ---------------------
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
-    plan_us = []
-    for k in range(args.plan_iters + 3):
-        flush.fill_(k & 0xFF)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        plan.balance_layer(0, ids)
-        b.record(stream)
-        b.synchronize()
-        if k >= 3:
-            plan_us.append(a.elapsed_time(b) * 1e3)
-    plan_us.sort()
-
-    # ---- staging alone ------------------------------------------------------
-    stage_ms = []
-    for k in range(6):
-        flush.fill_(k)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        plan.stage_replicas(0, native_w, slots)
-        b.record(stream)
-        b.synchronize()
-        if k >= 1:
-            stage_ms.append(a.elapsed_time(b))
+    plan_us = sorted(1e3 * t for t in _timed(torch, lambda: plan.balance_layer(0, ids),
+                                             args.plan_iters, stream, flush, skip=3))
+    stage_ms = _median(_timed(torch, lambda: plan.stage_replicas(0, native_w, slots), 5, stream, flush))
+    reduce_ms = _median(_timed(torch, lambda: plan.reduce_replica_grads(0, slot_grads, native_grads),
+                               5, stream, flush))
     n_rep = int(stats["replicas"])
-    view = plan.view(0)
-    rep_ptr = view["replica_expert_ptr"].cpu().numpy()
+    rep_ptr = plan.view(0)["replica_expert_ptr"].cpu().numpy()
     n_rep_exp = int((np.diff(rep_ptr) > 0).sum())
-    stage_bytes = (n_rep_exp + n_rep) * w.expert_elems * 2
-    stage_gbs = stage_bytes / (sum(stage_ms) / len(stage_ms) * 1e-3) / 1e9 if n_rep else 0.0
+    Wn = w.expert_elems
+    stage_bytes = (n_rep_exp + n_rep) * Wn * 2          # each replicated expert read once
+    reduce_bytes = n_rep_exp * Wn * 8 + n_rep * Wn * 4  # fp32 native in+out, bf16 replica in + zero
+    barrier()
 
     # ---- end to end through the public API with host buffers ---------------
     e2e = None
@@ -266,14 +290,11 @@ def run_gpu(args):
         e2e_ms = []
         for k in range(args.e2e_steps + 1):
             barrier()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
+            a, b = _events(torch)
             a.record(stream)
             ids.copy_(ids_h, non_blocking=True)
             hidden.copy_(hidden_h, non_blocking=True)
-            plan.balance_layer(0, ids)
-            plan.stage_replicas(0, native_w, slots)
-            plan.dispatch_layout(0, hidden, out=out)
+            step()
             st = plan.read_layer_stats(0)  # device -> host read of the step's result
             b.record(stream)
             b.synchronize()
@@ -294,6 +315,10 @@ def run_gpu(args):
         dist.destroy_process_group()
     if rank != 0:
         return None
+
+    del out, hidden, native_w, slots, slot_grads, native_grads
+    torch.cuda.empty_cache()
+    extras = measure_workloads(args, dev, flush) if args.extras else None
 
     peak, peak_kind = _peaks()
     perm_bytes = (w.N + rows_cap) * w.hidden * 2  # each token row read once, written per row
@@ -317,20 +342,20 @@ def run_gpu(args):
             "workload": f"{w.name}: Qwen3-235B-A22B-shaped MoE layer, R={w.R} simulated EP ranks, "
                         f"E={w.E}, top-{w.K}, T={w.T} tokens/rank, hidden {w.hidden} bf16, "
                         f"S={w.S} slot/rank of 3x{w.hidden}x{w.ffn} bf16, m={w.m}, Zipf s={w.zipf_s}",
-            "step": "ep_balance_layer + ep_stage_replicas + ep_dispatch_layout",
+            "step": ("forward: ep_balance_layer + ep_stage_replicas + ep_dispatch_layout; "
+                     "backward: ep_stage_replicas (re-stage from the cached plan) + "
+                     "ep_reduce_replica_grads (bf16 replica grads into fp32 native grads)"),
             "l2": "inputs larger than L2: each step's dispatch writes "
                   f"{rows_cap * w.hidden * 2 / 1e9:.1f} GB, evicting L2 between steps; "
-                  "plan latency measured after a 252 MiB L2 flush",
+                  "the per-piece timings flush L2 (252 MiB write) before every call",
             "parallelism": f"replicas x{world} (path does not shard)",
         },
-        "plan_us": {"median": plan_us[len(plan_us) // 2], "p90": plan_us[int(len(plan_us) * 0.9)],
+        "plan_us": {"median": _median(plan_us), "p90": plan_us[int(len(plan_us) * 0.9)],
                     "iters": len(plan_us)},
         "permute_gbs": achieved,
-        "stage_gbs": stage_gbs,
-        "max_mean_load": {"before": stats["before_max"] * w.R / A, "after": stats["after_max"] * w.R / A,
-                          "stop_reason": stats["stop_reason"],
-                          "tight_stop_reason": stats["tight_stop_reason"],
-                          "replicas": n_rep, "cap_idx": stats["cap_idx"]},
+        "stage_gbs": stage_bytes / (stage_ms * 1e-3) / 1e9 if n_rep else 0.0,
+        "reduce_gbs": reduce_bytes / (reduce_ms * 1e-3) / 1e9 if n_rep else 0.0,
+        "max_mean_load": _ratio(stats, w.R),
         "roofline": {"bound": "hbm", "kernel": "k_permute", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": perm_bytes,
@@ -338,10 +363,114 @@ def run_gpu(args):
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "workloads": extras,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return line
+
+
+def run_plan_only(args, w, ids, dev):
+    """ep_balance_layer alone (profiler captures of the plan kernels at full
+    size without the dispatch buffers)."""
+    import torch
+
+    from moe_expert_load_b200 import Plan, config_from_workload
+
+    plan = Plan(config_from_workload(w, num_layers=1), device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        plan.balance_layer(0, ids)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    us = sorted(1e3 * t for t in _timed(torch, lambda: plan.balance_layer(0, ids), args.plan_iters,
+                                        stream, flush, skip=0))
+    st = plan.read_layer_stats(0)
+    return {"mode": "plan-only", "workload": w.name, "plan_us_median": _median(us),
+            "max_mean_load": _ratio(st, w.R), "status": st["status"]}
+
+
+def measure_workloads(args, dev, flush):
+    """The other named workloads: plan latency and balance quality of each;
+    dispatch GB/s of dsv3 (with its Waterfill shared slot) and of stress (in
+    destination-rank windows, its output does not fit next to its input);
+    forward plans of the first sweep layers cached, then the backward re-stage
+    and gradient reduction replayed from the cache in reverse layer order."""
+    import numpy as np
+    import torch
+
+    from moe_expert_load_b200 import Plan, config_from_workload
+    from workloads import get_config, topk_ids
+
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name in ("tiny", "dsv3", "stress"):
+        w = get_config(name)
+        ids = torch.from_numpy(topk_ids(w)).to(dev)
+        plan = Plan(config_from_workload(w, num_layers=1), device=dev)
+        plan.balance_layer(0, ids)
+        st = plan.read_layer_stats(0)
+        pus = [1e3 * t for t in _timed(torch, lambda: plan.balance_layer(0, ids), 20, stream, flush, 3)]
+        entry = {"plan_us_median": _median(pus), "max_mean_load": _ratio(st, w.R), "rows": st["rows"]}
+        if name != "tiny":
+            g = torch.Generator(device=dev)
+            g.manual_seed(7)
+            hidden = torch.randn((w.N, w.hidden), generator=g, device=dev).to(torch.bfloat16)
+            rb = plan.view(0)["rank_row_begin"].cpu().numpy()
+            nwin = 1 if name == "dsv3" else 4
+            edges = [round(i * w.R / nwin) for i in range(nwin + 1)]
+            cap = max(int(rb[edges[i + 1]] - rb[edges[i]]) for i in range(nwin))
+            outw = torch.empty((cap, w.hidden), dtype=torch.bfloat16, device=dev)
+            win_bytes = 0
+            ids_np = ids.cpu().numpy()
+            dst = plan.view(0)["dst_row"].cpu().numpy().reshape(w.N, w.K)
+            srow = plan.view(0)["shared_row"]
+            srow = None if srow is None else srow.cpu().numpy().reshape(w.N)
+            for i in range(nwin):
+                lo, hi = int(rb[edges[i]]), int(rb[edges[i + 1]])
+                inwin = (dst >= lo) & (dst < hi)
+                loaded = inwin.any(axis=1)
+                if srow is not None:
+                    loaded |= (srow >= lo) & (srow < hi)
+                win_bytes += (int(loaded.sum()) + (hi - lo)) * w.hidden * 2
+            def dispatch_all():
+                for i in range(nwin):
+                    plan.dispatch_layout(0, hidden, out=outw, rank_begin=edges[i], rank_end=edges[i + 1])
+            ms = _median(_timed(torch, dispatch_all, 3, stream, flush))
+            entry["dispatch"] = {"windows": nwin, "bytes": win_bytes, "ms": ms,
+                                 "gbs": win_bytes / (ms * 1e-3) / 1e9}
+            del hidden, outw, ids_np
+        res[name] = entry
+        del plan, ids
+        torch.cuda.empty_cache()
+    # sweep: cached forward plans, then backward in reverse layer order
+    w = get_config("sweep")
+    L = args.sweep_layers
+    plan = Plan(config_from_workload(w, num_layers=w.layers), device=dev)
+    ids_l = [torch.from_numpy(topk_ids(w, l)).to(dev) for l in range(L)]
+    g = torch.Generator(device=dev)
+    g.manual_seed(9)
+    native_w = torch.randn((w.E, w.expert_elems), generator=g, device=dev).to(torch.bfloat16)
+    slots = torch.zeros((w.R, w.S, w.expert_elems), dtype=torch.bfloat16, device=dev)
+    slot_grads = torch.zeros_like(slots)
+    native_grads = torch.zeros((w.E, w.expert_elems), dtype=torch.float32, device=dev)
+    fwd_us, ratios, tight = [], [], []
+    for l in range(L):
+        fwd_us.append(1e3 * _timed(torch, lambda: plan.balance_layer(l, ids_l[l]), 1, stream, flush, 0)[0])
+        st = plan.read_layer_stats(l)
+        r = _ratio(st, w.R)
+        ratios.append(r["after"])
+        tight.append(r["tight_stop_reason"])
+    def backward():
+        for l in reversed(range(L)):
+            plan.stage_replicas(l, native_w, slots)
+            plan.reduce_replica_grads(l, slot_grads, native_grads)
+    bwd_ms = _median(_timed(torch, backward, 3, stream, flush))
+    ok = [r <= 1.05 or t == 1 for r, t in zip(ratios, tight)]
+    res["sweep"] = {"layers_measured": L, "plan_us_mean": float(np.mean(fwd_us)),
+                    "max_mean_after": {"mean": float(np.mean(ratios)), "max": float(np.max(ratios))},
+                    "layers_within_1.05_or_slot_limited": f"{sum(ok)}/{L}",
+                    "backward_ms_per_layer": bwd_ms / L}
+    return res
 
 
 def cpu_baseline(w, budget_s=15.0, steps=None):
@@ -427,6 +556,11 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the other workloads' measurements")
+    ap.add_argument("--sweep-layers", type=int, default=8)
+    ap.add_argument("--plan-only", action="store_true",
+                    help="time ep_balance_layer alone (for profiler captures)")
     ap.add_argument("--tokens-per-rank", type=int, default=None,
                     help="override T (small cases for profiler captures)")
     ap.add_argument("--ffn", type=int, default=None, help="override the expert FFN width")

@@ -24,10 +24,11 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
   // per layer (offset inside one layer block)
   size_t load, expert_total, W0, W, inst_expert, inst_quota, inst_off, rank_base, dst_row,
-      shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, stats;
+      shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, stats, tickets;
   size_t layer_bytes;
   // scratch (absolute)
-  size_t sub_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase;
+  size_t sub_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase,
+      shared_tot;
   size_t scratch_bytes;
   size_t total;
 };
@@ -83,8 +84,11 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   Layout L{};
   const size_t i4 = sizeof(int32_t);
   Bump b;
+  // stats, load, expert_total and tickets are contiguous: one memset clears them
+  L.stats = b.take(sizeof(ep_layer_stats));
   L.load = b.take(i4 * d.R * d.E);
   L.expert_total = b.take(i4 * d.E);
+  L.tickets = b.take(i4 * 4);
   L.W0 = b.take(i4 * d.R);
   L.W = b.take(i4 * d.R);
   L.inst_expert = b.take(i4 * d.R * d.G);
@@ -99,7 +103,6 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.rep_eptr = b.take(i4 * (d.E + 1));
   L.rep_nexp = b.take(i4);
   L.rep_experts = b.take(i4 * ((size_t)d.R * d.S + 1));
-  L.stats = b.take(sizeof(ep_layer_stats));
   L.layer_bytes = b.off;
   Bump s;
   s.off = L.layer_bytes * (size_t)num_layers;
@@ -113,6 +116,7 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.slack = s.take(i4 * d.R);
   L.wf = s.take(i4 * 2);
   L.sbase = s.take(i4 * d.R);
+  L.shared_tot = s.take(i4 * d.R);
   L.total = s.off;
   L.scratch_bytes = s.off - L.layer_bytes * (size_t)num_layers;
   return L;
@@ -143,6 +147,7 @@ ep::LayerBuf layer_buf(const ep_plan* p, int layer) {
   ep::LayerBuf L;
   L.load = at(p, b + l.load);
   L.expert_total = at(p, b + l.expert_total);
+  L.tickets = at(p, b + l.tickets);
   L.W0 = at(p, b + l.W0);
   L.W = at(p, b + l.W);
   L.inst_expert = at(p, b + l.inst_expert);
@@ -174,6 +179,7 @@ ep::Scratch scratch(const ep_plan* p) {
   s.slack = at(p, l.slack);
   s.wf = at(p, l.wf);
   s.sbase = at(p, l.sbase);
+  s.shared_tot = at(p, l.shared_tot);
   return s;
 }
 

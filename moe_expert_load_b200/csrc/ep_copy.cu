@@ -292,48 +292,84 @@ __global__ void __launch_bounds__(32) k_stage(StageArgs a) {
 constexpr int kReduceThreads = 256;
 constexpr int kReduceChunk = kReduceThreads * 8;
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Replica gradients are held raw (8 bf16 in one uint4, or 8 fp32 in two
+// float4) and converted at the add, to keep registers low enough for full
+// occupancy: the kernel is bound by how many bytes each SM keeps in flight.
+template <bool F32>
+struct Grad8 {
+  uint4 a, b;  // bf16: a only; fp32: a, b hold the bit patterns of 8 floats
+};
+
+template <bool F32>
+__device__ __forceinline__ Grad8<F32> load_grad8(const void* slot_grads, int64_t base) {
+  Grad8<F32> g;
+  if (F32) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(slot_grads) + base);
+    g.a = src[0];
+    g.b = src[1];
+  } else {
+    g.a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(slot_grads) + base);
+    g.b = make_uint4(0u, 0u, 0u, 0u);
+  }
+  return g;
+}
+
+template <bool F32>
+__device__ __forceinline__ void zero_grad8(void* slot_grads, int64_t base) {
+  if (F32) {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(slot_grads) + base);
+    dst[0] = make_uint4(0u, 0u, 0u, 0u);
+    dst[1] = make_uint4(0u, 0u, 0u, 0u);
+  } else {
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(slot_grads) + base) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// acc[i] = acc[i] + g[i], i = 0..7, one round-to-nearest fp32 add each.
+template <bool F32>
+__device__ __forceinline__ void add_grad8(float (&acc)[8], const Grad8<F32>& g) {
+  const uint32_t w[8] = {g.a.x, g.a.y, g.a.z, g.a.w, g.b.x, g.b.y, g.b.z, g.b.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  for (int i = 0; i < 8; ++i) {
+    const float v = F32 ? __uint_as_float(w[i])
+                        : __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
+    acc[i] = __fadd_rn(acc[i], v);
   }
 }
 
 template <bool F32>
-__global__ void __launch_bounds__(kReduceThreads)
+__global__ void __launch_bounds__(kReduceThreads, 4)
 k_reduce(const int32_t* __restrict__ rep_nexp, const int32_t* __restrict__ rep_experts,
          const int32_t* __restrict__ rep_eptr, const int32_t* __restrict__ rep_list,
-         void* __restrict__ slot_grads, float* __restrict__ native, int64_t Wn) {
-  const int64_t chunks = (Wn + kReduceChunk - 1) / kReduceChunk;
-  const int64_t total = (int64_t)rep_nexp[0] * chunks;
-  for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
-    const int64_t xi = t / chunks;
-    const int64_t j = (t - xi * chunks) * kReduceChunk + (int64_t)threadIdx.x * 8;
+         void* slot_grads, float* __restrict__ native, int64_t Wn) {
+  constexpr int kRepBatch = F32 ? 2 : 4;  // replica gradients loaded before any is cleared
+  const uint32_t chunks = (uint32_t)((Wn + kReduceChunk - 1) / kReduceChunk);
+  const uint32_t total = (uint32_t)rep_nexp[0] * chunks;
+  for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
+    const uint32_t xi = t / chunks;
+    const int64_t j = (int64_t)(t - xi * chunks) * kReduceChunk + (int64_t)threadIdx.x * 8;
     if (j >= Wn) continue;
     const int e = rep_experts[xi];
     const int p0 = rep_eptr[e], p1 = rep_eptr[e + 1];
     float4* nat = reinterpret_cast<float4*>(native + (int64_t)e * Wn + j);
     const float4 n0 = nat[0], n1 = nat[1];
     float acc[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-    for (int p = p0; p < p1; ++p) {
-      const int64_t base = (int64_t)rep_list[p] * Wn + j;
-      float g[8];
-      if (F32) {
-        float4* src = reinterpret_cast<float4*>(static_cast<float*>(slot_grads) + base);
-        const float4 g0 = src[0], g1 = src[1];
-        g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
-        g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
-        src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      } else {
-        uint4* src = reinterpret_cast<uint4*>(static_cast<uint16_t*>(slot_grads) + base);
-        bf16x8_to_f32(*src, g);
-        *src = make_uint4(0u, 0u, 0u, 0u);
+    for (int p = p0; p < p1; p += kRepBatch) {
+      // All loads of the batch are issued before any clearing store: a store
+      // through slot_grads may not be moved above a later load through it.
+      int64_t base[kRepBatch];
+      Grad8<F32> g[kRepBatch];
+#pragma unroll
+      for (int u = 0; u < kRepBatch; ++u) {
+        base[u] = p + u < p1 ? (int64_t)rep_list[p + u] * Wn + j : -1;
+        if (base[u] >= 0) g[u] = load_grad8<F32>(slot_grads, base[u]);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], g[i]);
+      for (int u = 0; u < kRepBatch; ++u)
+        if (base[u] >= 0) zero_grad8<F32>(slot_grads, base[u]);
+#pragma unroll
+      for (int u = 0; u < kRepBatch; ++u)  // instance order
+        if (base[u] >= 0) add_grad8<F32>(acc, g[u]);
     }
     nat[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     nat[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);

@@ -36,6 +36,7 @@ struct Dims {
 struct LayerBuf {
   int32_t* load;          // [R][E]
   int32_t* expert_total;  // [E]
+  int32_t* tickets;       // [4] arrival counters, zeroed with stats/load/expert_total
   int32_t* W0;            // [R]
   int32_t* W;             // [R]
   int32_t* inst_expert;   // [R][G]
@@ -65,6 +66,7 @@ struct Scratch {
   int32_t* slack;     // [R] Waterfill slack
   int32_t* wf;        // [2] Waterfill H, B
   int32_t* sbase;     // [R] first row of each rank's shared column
+  int32_t* shared_tot;  // [R] shared-slot rows per destination rank
 };
 
 // ---- native placement: contiguous balanced blocks ---------------------------

@@ -36,70 +36,72 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
   return z ^ (z >> 31);
 }
 
-// ---------------------------------------------------------------------------
-// a1: warp-aggregated histogram.  One warp per sub-chunk of kSubT tokens of one
-// source rank; lanes with equal ids are grouped with match.any and the group
-// leader adds the group size to the warp's private shared histogram.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
-k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, ep_layer_stats* stats) {
-  extern __shared__ int32_t sm_hist[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * kWarpsPerBlock + warp;
-  if (gw >= d.R * d.nsub) return;
-  int32_t* hist = sm_hist + warp * d.E;
-  for (int e = lane; e < d.E; e += 32) hist[e] = 0;
-  __syncwarp();
-  const int r = gw / d.nsub, sub = gw - (gw / d.nsub) * d.nsub;
-  const int t0 = sub * kSubT, t1 = min(d.T, t0 + kSubT);
-  const int32_t* src = ids + (int64_t)r * d.T * d.K;
-  const int a0 = t0 * d.K, a1 = t1 * d.K;
-  int bad = 0;
-  for (int a = a0; a < a1; a += 4 * 32) {
-    int v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int idx = a + u * 32 + lane;
-      v[u] = idx < a1 ? __ldg(src + idx) : -1;
-      if (idx < a1 && (v[u] < 0 || v[u] >= d.E)) { bad = 1; v[u] = -1; }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const unsigned peers = __match_any_sync(kFull, v[u]);
-      if (v[u] >= 0 && lane == __ffs(peers) - 1) hist[v[u]] += __popc(peers);
-      __syncwarp();
-    }
-  }
-  int32_t* out = s.sub_cnt + (int64_t)gw * d.E;
-  for (int e = lane; e < d.E; e += 32) out[e] = hist[e];
-  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&stats->status, EP_DEV_BAD_ID);
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor runs; pdl_wait() blocks until
+// the predecessor grid has completed and its writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// a1 (cont.): per (source rank, expert), exclusive scan of the sub-chunk counts
-// in token order (the bases of the stable ordinals) and the load-matrix entry.
-__global__ void __launch_bounds__(256) k_scan(Dims d, Scratch s, LayerBuf L) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= d.R * d.E) return;
-  const int r = i / d.E, e = i - (i / d.E) * d.E;
-  int32_t* p = s.sub_cnt + (int64_t)r * d.nsub * d.E + e;
-  int run = 0;
-  int sub = 0;
-  for (; sub + 8 <= d.nsub; sub += 8) {
-    int c[8];
+constexpr int kBatch = 16;  // ids per lane in flight
+
+// ---------------------------------------------------------------------------
+// a1: warp-aggregated histogram.  A block owns up to 8 consecutive sub-chunks
+// of kSubT tokens of one source rank, one per warp.  Lanes with equal ids are
+// grouped with match.any and the group leader adds the group size to the
+// warp's shared histogram; the warp writes its row of sub-chunk counts (the
+// bases of the stable ordinals, used by k_assign), and the block adds the sum
+// of its rows to the load matrix L[r][e] and the expert totals with integer
+// atomics (order-independent, so the result is deterministic).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, LayerBuf L) {
+  extern __shared__ int32_t sm_hist[];
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nbpr = (d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const int r = blockIdx.x / nbpr;
+  const int sub = (blockIdx.x - r * nbpr) * kWarpsPerBlock + warp;
+  const int E = d.E, K = d.K;
+  int32_t* hist = sm_hist + warp * E;
+  for (int e = lane; e < E; e += 32) hist[e] = 0;
+  __syncwarp();
+  int bad = 0;
+  if (sub < d.nsub) {
+    const int t0 = sub * kSubT, t1 = min(d.T, t0 + kSubT);
+    const int32_t* src = ids + (int64_t)r * d.T * K;
+    const int a1 = t1 * K;
+    for (int a = t0 * K; a < a1; a += kBatch * 32) {
+      int v[kBatch];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) c[u] = p[(int64_t)(sub + u) * d.E];
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = a + u * 32 + lane;
+        v[u] = idx < a1 ? __ldg(src + idx) : -1;
+        if (idx < a1 && (v[u] < 0 || v[u] >= E)) { bad = 1; v[u] = -1; }
+      }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      p[(int64_t)(sub + u) * d.E] = run;
-      run += c[u];
+      for (int u = 0; u < kBatch; ++u) {
+        if (a + u * 32 >= a1) break;
+        const unsigned peers = __match_any_sync(kFull, v[u]);
+        if (v[u] >= 0 && lane == __ffs(peers) - 1) hist[v[u]] += __popc(peers);
+        __syncwarp();
+      }
+    }
+    int32_t* out = s.sub_cnt + ((int64_t)r * d.nsub + sub) * E;
+    for (int e = lane; e < E; e += 32) out[e] = hist[e];
+  }
+  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&L.stats->status, EP_DEV_BAD_ID);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarpsPerBlock; ++w) c += sm_hist[w * E + e];
+    if (c) {
+      atomicAdd(&L.load[r * E + e], c);
+      atomicAdd(&L.expert_total[e], c);
     }
   }
-  for (; sub < d.nsub; ++sub) {
-    const int c = p[(int64_t)sub * d.E];
-    p[(int64_t)sub * d.E] = run;
-    run += c;
-  }
-  L.load[i] = run;
 }
 
 // ---------------------------------------------------------------------------
@@ -131,12 +133,9 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   const int warp = tid >> 5, lane = tid & 31;
   const int R = d.R, E = d.E, S = d.S, m = d.m;
 
-  for (int e = tid; e < E; e += nthr) {
-    int acc = 0;
-    for (int r = 0; r < R; ++r) acc += L.load[r * E + e];
-    Tot[e] = acc;
-    L.expert_total[e] = acc;
-  }
+  pdl_trigger();
+  pdl_wait();
+  for (int e = tid; e < E; e += nthr) Tot[e] = L.expert_total[e];
   if (tid == 0) s_iter_cap_hit = 0;
   __syncthreads();
   if (tid < R) {
@@ -437,6 +436,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   __shared__ int32_t s_ipq[kWarpsPerBlock][kMaxR];    // instance j: start of residual interval
   __shared__ int32_t s_iloc[kWarpsPerBlock][kMaxR];   // instance j: local take
   __shared__ int32_t s_jof[kWarpsPerBlock][kMaxR];    // rank -> instance j or -1
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * kWarpsPerBlock + warp;
   if (e >= d.E) return;
@@ -661,82 +662,191 @@ __device__ __forceinline__ int wf_pick(int r, int64_t token, const unsigned (&ma
 }
 
 // ---------------------------------------------------------------------------
-// a4 (+a5): token assignment.  One warp per sub-chunk.  The stable ordinal of
-// (t, k) among its source rank's assignments of expert e = exclusive base of
-// the sub-chunk + running count in the warp + rank inside the 32-lane group;
-// the ordinal selects the (source, expert) segment and thus the row.
+// a4 (+a5): token assignment.  A block owns up to 8 consecutive sub-chunks of
+// one source rank r (one per warp).  It first copies rank r's rerouting
+// segments into shared memory — for each expert, (first ordinal, row offset,
+// destination rank) — and the exclusive base of its first sub-chunk, the sum
+// of the rank's earlier sub-chunk counts.  The stable ordinal of (t, k) among
+// rank r's assignments of expert e = that base + the counts of the block's
+// earlier warps + the warp's running count + the rank inside the 32-lane
+// match.any group; the ordinal selects the segment and thus the row.
 // PASS 0: rows, no shared expert.  PASS 1: Waterfill picks, counted per
 // (destination rank, sub-chunk).  PASS 2: rows and shared-slot rows.
 // ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int seg_capacity(const Dims& d) {
+  // per source rank: at most one local segment per expert, and the remote
+  // overlaps of an expert are at most its number of instances
+  return 2 * d.E + d.R * d.S + 1;
+}
+
 template <int PASS>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   extern __shared__ int32_t sm[];
-  __shared__ int32_t s_rb[kMaxR + 1];
   __shared__ int32_t s_slack[kMaxR];
   __shared__ int32_t s_W[kMaxR];
   __shared__ int32_t s_sbase[kMaxR];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int32_t s_wsum[kWarpsPerBlock];
+  __shared__ int32_t s_total;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
   const int R = d.R, E = d.E, K = d.K;
-  for (int q = threadIdx.x; q <= R; q += blockDim.x) {
-    if (PASS != 1) s_rb[q] = L.rank_base[q];
-    if (PASS > 0 && q < R) {
+  const int nbpr = (d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const int r = blockIdx.x / nbpr;
+  const int sub0 = (blockIdx.x - r * nbpr) * kWarpsPerBlock;
+  const int sub = sub0 + warp;
+  const bool active = sub < d.nsub;
+  const int segcap = seg_capacity(d);
+  int32_t* sg_lo = sm;                                  // [E+1]
+  int32_t* sg_ord = sg_lo + E + 1;                      // [segcap] first ordinal
+  int32_t* sg_base = sg_ord + segcap;                   // [segcap] row - ordinal
+  int32_t* sg_rank = sg_base + segcap;                  // [segcap] destination rank
+  int32_t* base0 = sg_rank + (PASS > 0 ? segcap : 0);   // [E]
+  const int per_warp = E + (PASS > 0 ? R + (kSubT * K + 3) / 4 : 0);
+  int32_t* run = base0 + E + warp * per_warp;           // [E] running ordinals
+  int32_t* wrun = run + E;                              // [R] running shared ordinals
+  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);   // [kSubT*K] destination ranks
+
+  // The first batch of ids is an input no kernel of the plan writes: fetch it
+  // before waiting for the predecessor grid.
+  const int t0 = active ? sub * kSubT : 0, t1 = active ? min(d.T, t0 + kSubT) : 0;
+  const int a0 = t0 * K, a1 = t1 * K;
+  const int64_t rbase = (int64_t)r * d.T * K;
+  int v[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) {
+    const int idx = a0 + u * 32 + lane;
+    v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
+  }
+  pdl_trigger();
+  pdl_wait();
+
+  // rank r's segment table
+  {
+    const int per = (E + nthr - 1) / nthr;
+    const int eb = tid * per;
+    int cnt[4], s0[4], local = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = eb + u;
+      cnt[u] = 0;
+      s0[u] = 0;
+      if (u < per && e < E) {
+        const int sp = e * (R + 1) + r;
+        s0[u] = s.seg_ptr[sp];
+        cnt[u] = s.seg_ptr[sp + 1] - s0[u];
+      }
+      local += cnt[u];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int off = incl - local;
+    for (int w = 0; w < warp; ++w) off += s_wsum[w];
+    if (tid == nthr - 1) s_total = off + local;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = eb + u;
+      if (u < per && e < E) {
+        sg_lo[e] = off;
+        const int64_t gb = (int64_t)e * 3 * R + s0[u];
+        for (int j = 0; j < cnt[u] && off + j < segcap; ++j) {
+          const int ord = s.seg_ord[gb + j], rank = s.seg_rank[gb + j];
+          sg_ord[off + j] = ord;
+          if (PASS != 1) sg_base[off + j] = L.rank_base[rank] + s.seg_rel[gb + j] - ord;
+          if (PASS > 0) sg_rank[off + j] = rank;
+        }
+        off += cnt[u];
+      }
+    }
+  }
+  // exclusive base of the block's first sub-chunk
+  for (int e = tid; e < E; e += nthr) base0[e] = 0;
+  for (int q = tid; q < R; q += nthr) {
+    if (PASS > 0) {
       s_slack[q] = s.slack[q];
       s_W[q] = L.W[q];
       if (PASS == 2) s_sbase[q] = s.sbase[q];
     }
   }
   __syncthreads();
-  const int gw = blockIdx.x * kWarpsPerBlock + warp;
-  if (gw >= R * d.nsub) return;
-  // per-warp shared: run[E] | wrun[R] | dr[kSubT*K] (uint8)
-  const int per_warp = E + (PASS > 0 ? R + (kSubT * K + 3) / 4 : 0);
-  int32_t* run = sm + warp * per_warp;
-  int32_t* wrun = run + E;
-  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);
-  const int r = gw / d.nsub, sub = gw - (gw / d.nsub) * d.nsub;
-  const int32_t* base = s.sub_cnt + (int64_t)gw * E;
-  for (int e = lane; e < E; e += 32) run[e] = base[e];
-  __syncwarp();
-  const int t0 = sub * kSubT, t1 = min(d.T, t0 + kSubT);
-  const int a0 = t0 * K, a1 = t1 * K;
-  const int64_t rbase = (int64_t)r * d.T * K;
-  const int32_t* seg_ptr = s.seg_ptr;
-  for (int a = a0; a < a1; a += 32) {
-    const int idx = a + lane;
-    int e = -1;
-    if (idx < a1) {
-      e = __ldg(ids + rbase + idx);
-      if (e < 0 || e >= E) e = -1;
-    }
-    const unsigned peers = __match_any_sync(kFull, e);
-    const int rk = __popc(peers & lanemask_lt());
-    const int o = e >= 0 ? run[e] + rk : 0;
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) run[e] = o + __popc(peers);  // leader: rk = 0
-    __syncwarp();
-    if (idx < a1) {
-      int row = -1, rank = kNoRank;
-      if (e >= 0) {
-        const int sp = e * (R + 1) + r;
-        const int s0 = seg_ptr[sp], s1 = seg_ptr[sp + 1];
-        const int64_t sb = (int64_t)e * 3 * R;
-        int si = s1 - 1;
-        while (si > s0 && s.seg_ord[sb + si] > o) --si;
-        const int rk = (s1 > s0 && s0 >= 0 && s1 <= 3 * R) ? s.seg_rank[sb + si] : -1;
-        if (rk >= 0 && rk < R) {
-          rank = rk;
-          const int rel = s.seg_rel[sb + si] + (o - s.seg_ord[sb + si]);
-          if (PASS != 1) row = s_rb[rank] + rel;
-        } else {
-          atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
-        }
+  if (tid == 0) sg_lo[E] = s_total;
+  const bool overflow = s_total > segcap;
+  if (overflow) {
+    if (tid == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
+    return;
+  }
+  const int32_t* cnt_r = s.sub_cnt + (int64_t)r * d.nsub * E;
+  {
+    const int n = sub0 * E;
+    for (int i = tid; i < n; i += nthr * 8) {
+      int c[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int ii = i + u * nthr;
+        c[u] = ii < n ? cnt_r[ii] : 0;
       }
-      if (PASS != 1) L.dst_row[rbase + idx] = row;
-      if (PASS > 0) dr[idx - a0] = (uint8_t)rank;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int ii = i + u * nthr;
+        if (c[u]) atomicAdd(&base0[ii % E], c[u]);
+      }
     }
   }
+  __syncthreads();
+  if (!active) return;
+  for (int e = lane; e < E; e += 32) {
+    int acc = base0[e];
+    for (int w = 0; w < warp; ++w) acc += cnt_r[(int64_t)(sub0 + w) * E + e];
+    run[e] = acc;
+  }
+  __syncwarp();
+
+  bool inconsistent = false;
+  for (int a = a0; a < a1; a += kBatch * 32) {
+    if (a != a0) {
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = a + u * 32 + lane;
+        v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (a + u * 32 >= a1) break;
+      const int idx = a + u * 32 + lane;
+      const int e = (v[u] >= 0 && v[u] < E) ? v[u] : -1;
+      const unsigned peers = __match_any_sync(kFull, e);
+      const int rk = __popc(peers & lanemask_lt());
+      const int o = e >= 0 ? run[e] + rk : 0;
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) run[e] = o + __popc(peers);  // leader: rk = 0
+      __syncwarp();
+      if (idx < a1) {
+        int row = -1, rank = kNoRank;
+        if (e >= 0) {
+          const int lo = sg_lo[e], hi = sg_lo[e + 1];
+          int si = hi - 1;
+          while (si > lo && sg_ord[si] > o) --si;
+          if (hi > lo) {
+            if (PASS != 1) row = sg_base[si] + o;
+            if (PASS > 0) rank = sg_rank[si];
+          } else {
+            inconsistent = true;
+          }
+        }
+        if (PASS != 1) L.dst_row[rbase + idx] = row;
+        if (PASS > 0) dr[idx - a0] = (uint8_t)rank;
+      }
+    }
+  }
+  if (__any_sync(kFull, inconsistent) && lane == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
   if (PASS > 0) {
+    const int gw = r * d.nsub + sub;
     for (int q = lane; q < R; q += 32)
       wrun[q] = PASS == 1 ? 0 : s.wsub_cnt[(int64_t)q * R * d.nsub + gw];
     __syncwarp();
@@ -771,38 +881,67 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   }
 }
 
-// Shared-slot layout: for each destination rank c, exclusive scan of its pick
-// counts over (source rank, sub-chunk) — rows ordered by (source rank, token) —
-// then every rank's block = routed rows followed by its shared column.
-__global__ void __launch_bounds__(1024) k_shared_scan(Dims d, LayerBuf L, Scratch s) {
-  __shared__ int32_t s_tot[kMaxR];
+// Shared-slot layout: block c scans destination rank c's pick counts over
+// (source rank, sub-chunk) — rows ordered by (source rank, token) — in place;
+// the last block to finish (arrival ticket, no waiting) lays out every rank's
+// block: routed rows followed by its shared column.
+constexpr int kScanThreads = 256;
+constexpr int kScanItems = 8;
+
+__global__ void __launch_bounds__(kScanThreads) k_shared_scan(Dims d, LayerBuf L, Scratch s) {
+  __shared__ int32_t s_wsum[kScanThreads / 32];
+  __shared__ int32_t s_carry;
+  __shared__ int32_t s_last;
   __shared__ int32_t s_base[kMaxR + 1];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  pdl_trigger();
+  pdl_wait();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int R = d.R, G = d.G;
+  const int c = blockIdx.x;
   const int n = R * d.nsub;
-  for (int c = warp; c < R; c += nw) {
-    int32_t* col = s.wsub_cnt + (int64_t)c * n;
-    int carry = 0;
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      const int v = i < n ? col[i] : 0;
-      int incl = v;
+  int32_t* col = s.wsub_cnt + (int64_t)c * n;
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < n; b0 += kScanThreads * kScanItems) {
+    const int i0 = b0 + tid * kScanItems;
+    int v[kScanItems], local = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (i < n) col[i] = carry + incl - v;
-      carry += __shfl_sync(kFull, incl, 31);
+    for (int u = 0; u < kScanItems; ++u) {
+      v[u] = i0 + u < n ? col[i0 + u] : 0;
+      local += v[u];
     }
-    if (lane == 0) s_tot[c] = carry;
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int run = s_carry + incl - local;
+    for (int w = 0; w < warp; ++w) run += s_wsum[w];
+#pragma unroll
+    for (int u = 0; u < kScanItems; ++u) {
+      if (i0 + u < n) col[i0 + u] = run;
+      run += v[u];
+    }
+    __syncthreads();
+    if (tid == kScanThreads - 1) s_carry = run;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    s.shared_tot[c] = s_carry;
+    __threadfence();
+    s_last = atomicAdd(&L.tickets[0], 1) == R - 1;
   }
   __syncthreads();
+  if (!s_last) return;
+  __threadfence();
   if (warp == 0) {
     int carry = 0;
     for (int q0 = 0; q0 < R; q0 += 32) {
       const int q = q0 + lane;
-      const int v = q < R ? L.W[q] + s_tot[q] : 0;
+      const int v = q < R ? L.W[q] + s.shared_tot[q] : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -816,20 +955,20 @@ __global__ void __launch_bounds__(1024) k_shared_scan(Dims d, LayerBuf L, Scratc
   }
   __syncthreads();
   const int scol = d.Gmax + d.S;
-  for (int i = threadIdx.x; i < R * G; i += blockDim.x) {
-    const int q = i / G, col = i - (i / G) * G;
-    if (col == scol) {
-      L.inst_quota[i] = s_tot[q];
+  for (int i = tid; i < R * G; i += kScanThreads) {
+    const int q = i / G, cc = i - (i / G) * G;
+    if (cc == scol) {
+      L.inst_quota[i] = s.shared_tot[q];
       L.inst_off[i] = s_base[q] + L.W[q];
     } else {
       L.inst_off[i] = s_base[q] + s.inst_rel[i];
     }
   }
-  for (int q = threadIdx.x; q <= R; q += blockDim.x) {
+  for (int q = tid; q <= R; q += kScanThreads) {
     L.rank_base[q] = s_base[q];
     if (q < R) s.sbase[q] = s_base[q] + L.W[q];
   }
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     L.inst_off[R * G] = s_base[R];
     L.stats->rows = s_base[R];
   }
@@ -873,8 +1012,28 @@ k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
 size_t solve_smem(const Dims& d) { return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + d.E + 1); }
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
-  const int per_warp = d.E + (pass > 0 ? d.R + (kSubT * d.K + 3) / 4 : 0);
-  return sizeof(int32_t) * (size_t)kWarpsPerBlock * per_warp;
+  const size_t segcap = (size_t)seg_capacity(d);
+  const size_t per_warp = d.E + (pass > 0 ? d.R + (kSubT * d.K + 3) / 4 : 0);
+  return sizeof(int32_t) *
+         ((d.E + 1) + segcap * (pass > 0 ? 3 : 2) + d.E + (size_t)kWarpsPerBlock * per_warp);
+}
+
+// Launch with programmatic stream serialisation: the kernel may begin while
+// its predecessor in the stream is still running and waits for it in pdl_wait().
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 }  // namespace
@@ -895,26 +1054,34 @@ cudaError_t set_plan_attributes(int max_smem) {
 
 cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, const int32_t* ids,
                            cudaStream_t st) {
-  cudaError_t err = cudaMemsetAsync(L.stats, 0, sizeof(ep_layer_stats), st);
+  // stats, load matrix, expert totals and tickets are adjacent in the layer block
+  const size_t zero_bytes = reinterpret_cast<const char*>(L.tickets + 4) -
+                            reinterpret_cast<const char*>(L.stats);
+  cudaError_t err = cudaMemsetAsync(L.stats, 0, zero_bytes, st);
   if (err != cudaSuccess) return err;
-  const int nwarps = d.R * d.nsub;
-  const int nblk = (nwarps + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  if (nblk > 0) k_hist<<<nblk, kWarpsPerBlock * 32, hist_smem(d), st>>>(ids, d, s, L.stats);
-  k_scan<<<(d.R * d.E + 255) / 256, 256, 0, st>>>(d, s, L);
+  const unsigned nblk = (unsigned)(d.R * ((d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock));
+  const unsigned bt = kWarpsPerBlock * 32;
+  if (nblk > 0) k_hist<<<nblk, bt, hist_smem(d), st>>>(ids, d, s, L);
   const size_t ss = solve_smem(d);
-  const int sthreads = kMaxJ * 32;
-  if (d.S <= 1) k_solve<1><<<1, sthreads, ss, st>>>(d, L, s);
-  else if (d.S <= 2) k_solve<2><<<1, sthreads, ss, st>>>(d, L, s);
-  else if (d.S <= 4) k_solve<4><<<1, sthreads, ss, st>>>(d, L, s);
-  else k_solve<8><<<1, sthreads, ss, st>>>(d, L, s);
-  k_reroute<<<(d.E + kWarpsPerBlock - 1) / kWarpsPerBlock, kWarpsPerBlock * 32, 0, st>>>(d, L, s);
+  const unsigned sthreads = kMaxJ * 32;
+  if (d.S <= 1) err = launch_pdl(k_solve<1>, 1, sthreads, ss, st, d, L, s);
+  else if (d.S <= 2) err = launch_pdl(k_solve<2>, 1, sthreads, ss, st, d, L, s);
+  else if (d.S <= 4) err = launch_pdl(k_solve<4>, 1, sthreads, ss, st, d, L, s);
+  else err = launch_pdl(k_solve<8>, 1, sthreads, ss, st, d, L, s);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(k_reroute, (unsigned)((d.E + kWarpsPerBlock - 1) / kWarpsPerBlock), bt, 0, st, d,
+                   L, s);
+  if (err != cudaSuccess) return err;
   if (!d.sh) {
-    if (nblk > 0) k_assign<0><<<nblk, kWarpsPerBlock * 32, assign_smem(d, 0), st>>>(ids, d, L, s);
+    if (nblk > 0) err = launch_pdl(k_assign<0>, nblk, bt, assign_smem(d, 0), st, ids, d, L, s);
   } else {
-    if (nblk > 0) k_assign<1><<<nblk, kWarpsPerBlock * 32, assign_smem(d, 1), st>>>(ids, d, L, s);
-    k_shared_scan<<<1, 1024, 0, st>>>(d, L, s);
-    if (nblk > 0) k_assign<2><<<nblk, kWarpsPerBlock * 32, assign_smem(d, 2), st>>>(ids, d, L, s);
+    if (nblk > 0) err = launch_pdl(k_assign<1>, nblk, bt, assign_smem(d, 1), st, ids, d, L, s);
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(k_shared_scan, (unsigned)d.R, kScanThreads, 0, st, d, L, s);
+    if (err != cudaSuccess) return err;
+    if (nblk > 0) err = launch_pdl(k_assign<2>, nblk, bt, assign_smem(d, 2), st, ids, d, L, s);
   }
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

@@ -22,7 +22,13 @@ namespace ep {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kStages = 4;                  // row / tile buffers per CTA
+#ifndef EP_COPY_STAGES
+#define EP_COPY_STAGES 4
+#endif
+#ifndef EP_PERMUTE_SMEM_BUDGET
+#define EP_PERMUTE_SMEM_BUDGET (200 * 1024)
+#endif
+constexpr int kStages = EP_COPY_STAGES;     // row / tile buffers per CTA
 constexpr uint32_t kWaitSpins = 1u << 20;   // try_wait polls before giving up
 constexpr int kStageTile = 16384;           // bytes per staging tile
 
@@ -290,95 +296,120 @@ __global__ void __launch_bounds__(32) k_stage(StageArgs a) {
 // are zeroed.
 // ---------------------------------------------------------------------------
 constexpr int kReduceThreads = 256;
-constexpr int kReduceChunk = kReduceThreads * 8;
 
-// Replica gradients are held raw (8 bf16 in one uint4, or 8 fp32 in two
-// float4) and converted at the add, to keep registers low enough for full
-// occupancy: the kernel is bound by how many bytes each SM keeps in flight.
+// The replica lists of the layer (at most R*S slots) are staged in shared
+// memory once per block, so the streaming loops have no dependent global
+// lookups.  Clearing a replica gradient in the thread that has just loaded it
+// stalls the load/store pipeline on the in-flight line (measured: ~1.1 TB/s);
+// so k_reduce only loads replica gradients, and k_clear_replicas zeroes them
+// afterwards (together ~6 TB/s).
+constexpr int kMaxRepSlots = kMaxR * kMaxS;
+
+struct RepTables {
+  int32_t exp[kMaxRepSlots];      // replicated expert i
+  int32_t ptr[kMaxRepSlots + 1];  // its replicas: slot[ptr[i] .. ptr[i+1])
+  int32_t slot[kMaxRepSlots];     // slot index q*S + s, instance order
+};
+
+__device__ __forceinline__ int stage_rep_tables(RepTables& t, const int32_t* rep_nexp,
+                                                const int32_t* rep_experts, const int32_t* rep_eptr,
+                                                const int32_t* rep_list, int E) {
+  const int nexp = rep_nexp[0];
+  for (int i = threadIdx.x; i < nexp; i += blockDim.x) {
+    const int e = rep_experts[i];
+    t.exp[i] = e;
+    t.ptr[i] = rep_eptr[e];
+  }
+  const int nrep = rep_eptr[E];
+  if (threadIdx.x == 0) t.ptr[nexp] = nrep;
+  for (int i = threadIdx.x; i < nrep; i += blockDim.x) t.slot[i] = rep_list[i];
+  __syncthreads();
+  return nexp;
+}
+
+// 8 gradient values of one replica: bf16 in one 16-byte word, fp32 in two.
 template <bool F32>
-struct Grad8 {
-  uint4 a, b;  // bf16: a only; fp32: a, b hold the bit patterns of 8 floats
+struct Raw8 {
+  uint4 a, b;
 };
 
 template <bool F32>
-__device__ __forceinline__ Grad8<F32> load_grad8(const void* slot_grads, int64_t base) {
-  Grad8<F32> g;
+__device__ __forceinline__ Raw8<F32> load8(const void* g, int64_t base) {
+  Raw8<F32> r;
   if (F32) {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(slot_grads) + base);
-    g.a = src[0];
-    g.b = src[1];
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(g) + base);
+    r.a = p[0];
+    r.b = p[1];
   } else {
-    g.a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(slot_grads) + base);
-    g.b = make_uint4(0u, 0u, 0u, 0u);
+    r.a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g) + base);
+    r.b = r.a;
   }
-  return g;
+  return r;
 }
 
 template <bool F32>
-__device__ __forceinline__ void zero_grad8(void* slot_grads, int64_t base) {
-  if (F32) {
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(slot_grads) + base);
-    dst[0] = make_uint4(0u, 0u, 0u, 0u);
-    dst[1] = make_uint4(0u, 0u, 0u, 0u);
-  } else {
-    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(slot_grads) + base) = make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
-// acc[i] = acc[i] + g[i], i = 0..7, one round-to-nearest fp32 add each.
-template <bool F32>
-__device__ __forceinline__ void add_grad8(float (&acc)[8], const Grad8<F32>& g) {
-  const uint32_t w[8] = {g.a.x, g.a.y, g.a.z, g.a.w, g.b.x, g.b.y, g.b.z, g.b.w};
+__device__ __forceinline__ void add8(float (&acc)[8], const Raw8<F32>& r) {
+  const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float v = F32 ? __uint_as_float(w[i])
                         : __uint_as_float((i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16));
-    acc[i] = __fadd_rn(acc[i], v);
+    acc[i] = __fadd_rn(acc[i], v);  // instance order, one round-to-nearest add each
   }
 }
 
 template <bool F32>
-__global__ void __launch_bounds__(kReduceThreads, 4)
+__global__ void __launch_bounds__(kReduceThreads)
 k_reduce(const int32_t* __restrict__ rep_nexp, const int32_t* __restrict__ rep_experts,
          const int32_t* __restrict__ rep_eptr, const int32_t* __restrict__ rep_list,
-         void* slot_grads, float* __restrict__ native, int64_t Wn) {
-  constexpr int kRepBatch = F32 ? 2 : 4;  // replica gradients loaded before any is cleared
-  const uint32_t chunks = (uint32_t)((Wn + kReduceChunk - 1) / kReduceChunk);
-  const uint32_t total = (uint32_t)rep_nexp[0] * chunks;
-  for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
-    const uint32_t xi = t / chunks;
-    const int64_t j = (int64_t)(t - xi * chunks) * kReduceChunk + (int64_t)threadIdx.x * 8;
-    if (j >= Wn) continue;
-    const int e = rep_experts[xi];
-    const int p0 = rep_eptr[e], p1 = rep_eptr[e + 1];
+         const void* __restrict__ slot_grads, float* __restrict__ native, int64_t Wn, int E) {
+  constexpr int kB = F32 ? 4 : 8;  // replica loads issued together
+  __shared__ RepTables t;
+  const int nexp = stage_rep_tables(t, rep_nexp, rep_experts, rep_eptr, rep_list, E);
+  const uint32_t vpe = (uint32_t)(Wn / 8);
+  const uint32_t total = (uint32_t)nexp * vpe;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t v = blockIdx.x * blockDim.x + threadIdx.x; v < total; v += stride) {
+    const uint32_t xi = v / vpe;
+    const int64_t j = (int64_t)(v - xi * vpe) * 8;
+    const int e = t.exp[xi];
+    const int p0 = t.ptr[xi], p1 = t.ptr[xi + 1];
     float4* nat = reinterpret_cast<float4*>(native + (int64_t)e * Wn + j);
     const float4 n0 = nat[0], n1 = nat[1];
     float acc[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-    for (int p = p0; p < p1; p += kRepBatch) {
-      // All loads of the batch are issued before any clearing store: a store
-      // through slot_grads may not be moved above a later load through it.
-      int64_t base[kRepBatch];
-      Grad8<F32> g[kRepBatch];
+    for (int p = p0; p < p1; p += kB) {
+      Raw8<F32> r[kB];
 #pragma unroll
-      for (int u = 0; u < kRepBatch; ++u) {
-        base[u] = p + u < p1 ? (int64_t)rep_list[p + u] * Wn + j : -1;
-        if (base[u] >= 0) g[u] = load_grad8<F32>(slot_grads, base[u]);
-      }
+      for (int u = 0; u < kB; ++u)
+        if (p + u < p1) r[u] = load8<F32>(slot_grads, (int64_t)t.slot[p + u] * Wn + j);
 #pragma unroll
-      for (int u = 0; u < kRepBatch; ++u)
-        if (base[u] >= 0) zero_grad8<F32>(slot_grads, base[u]);
-#pragma unroll
-      for (int u = 0; u < kRepBatch; ++u)  // instance order
-        if (base[u] >= 0) add_grad8<F32>(acc, g[u]);
+      for (int u = 0; u < kB; ++u)
+        if (p + u < p1) add8<F32>(acc, r[u]);
     }
     nat[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     nat[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
+// Zero every filled replica slot's gradient (16-byte stores).
+__global__ void __launch_bounds__(kReduceThreads)
+k_clear_replicas(const int32_t* __restrict__ rep_nexp, const int32_t* __restrict__ rep_experts,
+                 const int32_t* __restrict__ rep_eptr, const int32_t* __restrict__ rep_list,
+                 uint4* slot_grads, int64_t slot_words, int E) {
+  __shared__ RepTables t;
+  stage_rep_tables(t, rep_nexp, rep_experts, rep_eptr, rep_list, E);
+  const int nrep = rep_eptr[E];
+  const uint64_t total = (uint64_t)nrep * (uint64_t)slot_words;
+  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+  for (uint64_t w = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += stride) {
+    const uint64_t p = w / (uint64_t)slot_words;
+    slot_grads[(uint64_t)t.slot[p] * slot_words + (w - p * slot_words)] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 int permute_ctas_per_sm(uint32_t row_bytes) {
   const size_t smem = 128 + (size_t)kStages * row_bytes;
-  int c = (int)((200u * 1024u) / smem);
+  int c = (int)((size_t)EP_PERMUTE_SMEM_BUDGET / smem);
   if (c > 16) c = 16;
   if (c < 1) c = 1;
   return c;
@@ -436,13 +467,23 @@ cudaError_t launch_stage(const Dims& d, const LayerBuf& L, const void* native_w,
 cudaError_t launch_reduce(const Dims& d, const LayerBuf& L, void* slot_grads, int grad_f32,
                           float* native_grads, int num_sms, cudaStream_t st) {
   if (d.Wn == 0 || d.S == 0) return cudaSuccess;
-  const unsigned grid = (unsigned)(num_sms * 8);
+  int per_sm = 0;
+  cudaError_t e = grad_f32 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_reduce<true>,
+                                                                          kReduceThreads, 0)
+                           : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_reduce<false>,
+                                                                          kReduceThreads, 0);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(num_sms * (per_sm > 0 ? per_sm : 1));
   if (grad_f32)
     k_reduce<true><<<grid, kReduceThreads, 0, st>>>(L.rep_nexp, L.rep_experts, L.rep_eptr,
-                                                    L.rep_list, slot_grads, native_grads, d.Wn);
+                                                    L.rep_list, slot_grads, native_grads, d.Wn, d.E);
   else
     k_reduce<false><<<grid, kReduceThreads, 0, st>>>(L.rep_nexp, L.rep_experts, L.rep_eptr,
-                                                     L.rep_list, slot_grads, native_grads, d.Wn);
+                                                     L.rep_list, slot_grads, native_grads, d.Wn, d.E);
+  const int64_t slot_words = d.Wn * (grad_f32 ? 4 : 2) / 16;
+  k_clear_replicas<<<(unsigned)(num_sms * 4), kReduceThreads, 0, st>>>(
+      L.rep_nexp, L.rep_experts, L.rep_eptr, L.rep_list, static_cast<uint4*>(slot_grads), slot_words,
+      d.E);
   return cudaGetLastError();
 }
 

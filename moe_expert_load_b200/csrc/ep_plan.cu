@@ -47,10 +47,10 @@ __device__ __forceinline__ void pdl_trigger() {
 constexpr int kBatch = 16;  // ids per lane in flight
 
 // ---------------------------------------------------------------------------
-// a1: warp-aggregated histogram.  A block owns up to 8 consecutive sub-chunks
-// of kSubT tokens of one source rank, one per warp.  Lanes with equal ids are
-// grouped with match.any and the group leader adds the group size to the
-// warp's shared histogram; the warp writes its row of sub-chunk counts (the
+// a1: load histogram.  A block owns up to 8 consecutive sub-chunks of kSubT
+// tokens of one source rank, one per warp.  Each warp counts its sub-chunk into
+// a private shared-memory histogram with shared atomic adds (16 ids per lane in
+// flight, no dependence between rounds); the warp writes its row of counts (the
 // bases of the stable ordinals, used by k_assign), and the block adds the sum
 // of its rows to the load matrix L[r][e] and the expert totals with integer
 // atomics (order-independent, so the result is deterministic).
@@ -81,13 +81,10 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, LayerBuf L) {
         if (idx < a1 && (v[u] < 0 || v[u] >= E)) { bad = 1; v[u] = -1; }
       }
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        if (a + u * 32 >= a1) break;
-        const unsigned peers = __match_any_sync(kFull, v[u]);
-        if (v[u] >= 0 && lane == __ffs(peers) - 1) hist[v[u]] += __popc(peers);
-        __syncwarp();
-      }
+      for (int u = 0; u < kBatch; ++u)
+        if (v[u] >= 0) atomicAdd(&hist[v[u]], 1);  // integer: order-independent
     }
+    __syncwarp();
     int32_t* out = s.sub_cnt + ((int64_t)r * d.nsub + sub) * E;
     for (int e = lane; e < E; e += 32) out[e] = hist[e];
   }

@@ -68,6 +68,8 @@ def _load():
         lib.orc_waterfill.restype = ctypes.c_int
         lib.orc_permute.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int64, P, P, P, P]
         lib.orc_permute.restype = None
+        lib.orc_combine.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P]
+        lib.orc_combine.restype = None
         lib.orc_stage.argtypes = [ctypes.c_int32] * 4 + [P, ctypes.c_int64, P, P]
         lib.orc_stage.restype = None
         lib.orc_reduce_grads.argtypes = [ctypes.c_int32] * 4 + [P, ctypes.c_int64, ctypes.c_int32, P, P]
@@ -218,6 +220,21 @@ def permute_range(p: Plan, hidden_rows: np.ndarray, n0: int, out: np.ndarray) ->
     dst = np.ascontiguousarray(p.dst_row.reshape(-1, p.K)[n0:n0 + n])
     srow = None if p.shared_row is None else np.ascontiguousarray(p.shared_row.reshape(-1)[n0:n0 + n])
     _load().orc_permute(n, p.K, hidden_rows.strides[0], _p(hidden_rows), _p(dst), _p(srow), _p(out))
+
+
+def combine(p: Plan, expert_out: np.ndarray, weights: np.ndarray) -> np.ndarray:
+    """fp64 combine: gate-weighted sum of each token's routed rows, plus its
+    shared-expert row with weight 1.  expert_out: bf16 bits (uint16) [rows][H];
+    weights: float32 [R][T][K].  Returns float64 [N][H]."""
+    x = np.ascontiguousarray(expert_out, dtype=np.uint16)
+    H = x.shape[1]
+    N = p.R * p.T
+    dst = np.ascontiguousarray(p.dst_row.reshape(N, p.K), dtype=np.int64)
+    wt = np.ascontiguousarray(weights.reshape(N, p.K), dtype=np.float32)
+    srow = None if p.shared_row is None else np.ascontiguousarray(p.shared_row.reshape(N), dtype=np.int64)
+    out = np.zeros((N, H), np.float64)
+    _load().orc_combine(N, p.K, H, _p(x), _p(dst), _p(wt), _p(srow), _p(out))
+    return out
 
 
 def stage(p: Plan, native_w: np.ndarray, slots: np.ndarray) -> None:

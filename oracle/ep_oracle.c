@@ -571,6 +571,34 @@ void orc_permute(int64_t N, int32_t K, int64_t row_bytes, const uint8_t* hidden,
   }
 }
 
+/* ---- combine (reverse of the dispatch, with gate weights) -------------- */
+/* After expert compute each dispatch row holds its expert's output for one
+ * (token, k) (or the shared expert's output for the token).  The token's
+ * output is the gate-weighted sum of its routed rows plus its shared-expert
+ * row with weight 1 (the shared expert is not gated), computed here exactly
+ * enough in fp64: out[n][h] = sum_k w[n][k] * x[dst_row[n][k]][h]
+ * (+ x[shared_row[n]][h]); rows of -1 (dropped ids) contribute nothing. */
+static double bf16_to_f64(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+void orc_combine(int64_t N, int32_t K, int32_t H, const uint16_t* x, const int64_t* dst_row,
+                 const float* w, const int64_t* shared_row, double* out) {
+  for (int64_t n = 0; n < N; ++n)
+    for (int32_t h = 0; h < H; ++h) {
+      double acc = 0.0;
+      for (int32_t k = 0; k < K; ++k) {
+        const int64_t d = dst_row[n * K + k];
+        if (d >= 0) acc += (double)w[n * K + k] * bf16_to_f64(x[d * H + h]);
+      }
+      if (shared_row) acc += bf16_to_f64(x[shared_row[n] * H + h]);
+      out[n * H + h] = acc;
+    }
+}
+
 /* ---- O11: stage replica weights (bit copy) ----------------------------- */
 void orc_stage(int32_t R, int32_t S, int32_t G, int32_t Gmax, const int32_t* inst_expert,
                int64_t elem_bytes, const uint8_t* native_w, uint8_t* slots) {

@@ -438,3 +438,58 @@ def test_reduce_grads_is_sequential_fp32_sum(grad_dtype):
     assert (gg[filled] == 0).all()
     assert (gg[~filled] == g[~filled]).all()
     assert p.replicas > 0
+
+
+# ---- combine (reverse of the dispatch) -------------------------------------------
+def _bf16_bits(a):
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    return ((u + ((u >> 16) & 1) + 0x7FFF) >> 16).astype(np.uint16)
+
+
+def _bits_f64(b):
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("shared", [False, True])
+def test_combine_is_adjoint_of_dispatch(shared):
+    # dispatching hidden rows and combining them back with gate weights w gives
+    # (sum_k w_k + [shared]) * hidden exactly (each dispatch row is a copy)
+    cfg = get_config("tiny").replace(shared_expert=shared)
+    ids = topk_ids(cfg)
+    p = _plan_cfg(cfg, ids)
+    rng = np.random.default_rng(12)
+    hidden = _bf16_bits(rng.standard_normal((cfg.N, cfg.hidden)))
+    x = oracle.permute(p, hidden)
+    w = rng.random((cfg.R, cfg.T, cfg.K)).astype(np.float32)
+    y = oracle.combine(p, x, w)
+    scale = w.reshape(cfg.N, cfg.K).astype(np.float64).sum(1) + (1.0 if shared else 0.0)
+    np.testing.assert_allclose(y, scale[:, None] * _bits_f64(hidden), rtol=1e-14, atol=0)
+
+
+def test_combine_is_linear_and_skips_dropped_rows():
+    cfg = get_config("tiny")
+    ids = topk_ids(cfg).copy()
+    ids[1, 10, 0] = -1  # dropped id: its weight must not matter
+    p = _plan_cfg(cfg, ids)
+    rng = np.random.default_rng(13)
+    xa = _bf16_bits(rng.standard_normal((p.rows, 16)))
+    xb = _bf16_bits(rng.standard_normal((p.rows, 16)))
+    w = rng.random((cfg.R, cfg.T, cfg.K)).astype(np.float32)
+    ya, yb = oracle.combine(p, xa, w), oracle.combine(p, xb, w)
+    # linear in the gate weights: doubling w doubles the output exactly
+    np.testing.assert_array_equal(oracle.combine(p, xa, 2 * w), 2 * ya)
+    w2 = w.copy()
+    w2[1, 10, 0] = 1e6
+    np.testing.assert_array_equal(oracle.combine(p, xa, w2), ya)
+    # all-ones expert outputs: each token gets the sum of the weights of its valid ids
+    ones = _bf16_bits(np.ones((p.rows, 16)))
+    valid = (np.asarray(ids) >= 0).reshape(-1, cfg.K)
+    expect = (w.reshape(-1, cfg.K).astype(np.float64) * valid).sum(1)
+    np.testing.assert_allclose(oracle.combine(p, ones, w), np.repeat(expect[:, None], 16, 1), rtol=1e-14)
+    # additive in the expert outputs (exact sums of small integers)
+    xi = _bf16_bits(rng.integers(-8, 8, size=(p.rows, 16)).astype(np.float64))
+    xj = _bf16_bits(rng.integers(-8, 8, size=(p.rows, 16)).astype(np.float64))
+    xij = _bf16_bits(_bits_f64(xi) + _bits_f64(xj))
+    wi = np.ones_like(w)
+    np.testing.assert_array_equal(oracle.combine(p, xij, wi), oracle.combine(p, xi, wi) + oracle.combine(p, xj, wi))
+    assert yb.shape == ya.shape

@@ -274,6 +274,13 @@ def run_gpu(args):
     stage_ms = _median(_timed(torch, lambda: plan.stage_replicas(0, native_w, slots), 5, stream, flush))
     reduce_ms = _median(_timed(torch, lambda: plan.reduce_replica_grads(0, slot_grads, native_grads),
                                5, stream, flush))
+    # combine (reverse of the dispatch; not part of the step): the dispatch
+    # output stands in for the expert outputs, bf16 result per token
+    gate_w = torch.rand((w.R, w.T, w.K), generator=g, device=dev)
+    y = torch.empty((w.N, w.hidden), dtype=torch.bfloat16, device=dev)
+    combine_ms = _median(_timed(torch, lambda: plan.combine(0, out, gate_w, out=y), 5, stream, flush))
+    combine_bytes = (rows_cap + w.N) * w.hidden * 2 + w.N * w.K * 8
+    del y
     n_rep = int(stats["replicas"])
     rep_ptr = plan.view(0)["replica_expert_ptr"].cpu().numpy()
     n_rep_exp = int((np.diff(rep_ptr) > 0).sum())
@@ -355,6 +362,7 @@ def run_gpu(args):
         "permute_gbs": achieved,
         "stage_gbs": stage_bytes / (stage_ms * 1e-3) / 1e9 if n_rep else 0.0,
         "reduce_gbs": reduce_bytes / (reduce_ms * 1e-3) / 1e9 if n_rep else 0.0,
+        "combine_gbs": combine_bytes / (combine_ms * 1e-3) / 1e9,
         "max_mean_load": _ratio(stats, w.R),
         "roofline": {"bound": "hbm", "kernel": "k_permute", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,

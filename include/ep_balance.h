@@ -216,6 +216,24 @@ EP_API ep_status_t ep_reduce_replica_grads(ep_plan* plan, int32_t layer, void* d
                                     int32_t grad_dtype, float* d_native_grads, void* stream);
 
 /*
+ * Combine, the reverse of ep_dispatch_layout ([W] §"Shared expert fusion":
+ * routed and shared experts share one dispatch -> grouped GEMM -> combine
+ * flow; [U]: dispatch by the rerouting plan): after expert compute, dispatch
+ * row i of d_expert_out [rows][hidden] bf16 holds its expert's output for the
+ * (token, k) that was sent there.  For every token n = r*T + t:
+ *   out[n] = sum over k ascending of w[r][t][k] * x[dst_row[r][t][k]]
+ *            (+ x[shared_row[r][t]] with weight 1 when the layer has a shared
+ *            expert),
+ * accumulated in fp32, one fused multiply-add per k in ascending k, the shared
+ * row added last; rows of dropped ids (-1) contribute nothing.  d_weights
+ * [R][T][K] fp32 (the gate's top-k weights); d_out [R*T][hidden] of out_dtype
+ * (0 = bf16, round to nearest even; 1 = fp32).  All buffers 16-byte aligned.
+ */
+EP_API ep_status_t ep_combine(ep_plan* plan, int32_t layer, const void* d_expert_out,
+                              const float* d_weights, void* d_out, int32_t out_dtype,
+                              void* stream);
+
+/*
  * Standalone Waterfill ([W] §"Waterfill"): for routed per-rank loads d_load [R]
  * (int32) and the destination rank of every routed assignment d_dst_rank
  * [R][T][K] (int32, -1 = none), pick each token's shared-expert rank:

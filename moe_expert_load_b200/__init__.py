@@ -169,6 +169,22 @@ class Plan:
             self.handle, layer, _ptr(hidden), _ptr(out), out.shape[0], rank_begin, rank_end, _stream(stream)))
         return out
 
+    def combine(self, layer: int, expert_out: torch.Tensor, weights: torch.Tensor,
+                out: Optional[torch.Tensor] = None, out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+        """ep_combine: gate-weighted sum of each token's dispatch rows (+ shared row)."""
+        if weights.dtype != torch.float32 or tuple(weights.shape) != (self.R, self.T, self.K):
+            raise ValueError(f"weights must be float32 [{self.R}, {self.T}, {self.K}]")
+        out = _combine_out(self, expert_out, out, out_dtype)
+        if out.dtype == torch.bfloat16:
+            dt = 0
+        elif out.dtype == torch.float32:
+            dt = 1
+        else:
+            raise ValueError("out must be bfloat16 or float32")
+        _check("ep_combine", self.lib.ep_combine(
+            self.handle, layer, _ptr(expert_out), _ptr(weights), _ptr(out), dt, _stream(stream)))
+        return out
+
     def stage_replicas(self, layer: int, native_w: torch.Tensor, slots: torch.Tensor, stream=None) -> None:
         """ep_stage_replicas: native_w bf16 [E][Wn] -> slots bf16 [R][S][Wn]."""
         _check("ep_stage_replicas", self.lib.ep_stage_replicas(
@@ -187,6 +203,12 @@ class Plan:
             raise ValueError("slot_grads must be bfloat16 or float32")
         _check("ep_reduce_replica_grads", self.lib.ep_reduce_replica_grads(
             self.handle, layer, _ptr(slot_grads), dt, _ptr(native_grads), _stream(stream)))
+
+
+def _combine_out(plan, expert_out, out, out_dtype):
+    if out is None:
+        out = torch.empty((plan.R * plan.T, expert_out.shape[1]), dtype=out_dtype, device=expert_out.device)
+    return out
 
 
 def ep_waterfill(load: torch.Tensor, dst_rank: torch.Tensor, seed: int, bonus_permille: int = 10,

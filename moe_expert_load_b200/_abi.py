@@ -27,7 +27,7 @@ EXPORTS = (
     "ep_plan_workspace_bytes", "ep_plan_create", "ep_plan_destroy", "ep_balance_layer",
     "ep_layer_view_get", "ep_read_layer_stats", "ep_dispatch_layout", "ep_stage_replicas",
     "ep_reduce_replica_grads", "ep_waterfill", "ep_status_string", "ep_abi_version",
-    "ep_load_matrix_static",
+    "ep_load_matrix_static", "ep_combine",
 )
 
 
@@ -103,6 +103,7 @@ def load():
         "ep_stage_replicas": (S, [P, I32, P, P, P]),
         "ep_reduce_replica_grads": (S, [P, I32, P, I32, P, P]),
         "ep_waterfill": (S, [I32, I32, I32, P, P, ctypes.c_uint64, I32, P, P, P]),
+        "ep_combine": (S, [P, I32, P, P, P, I32, P]),
         "ep_status_string": (ctypes.c_char_p, [S]),
         "ep_abi_version": (I32, []),
     }

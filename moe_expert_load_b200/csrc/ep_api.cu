@@ -333,6 +333,22 @@ ep_status_t ep_dispatch_layout(ep_plan* plan, int32_t layer, const void* d_hidde
                                          plan->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
+ep_status_t ep_combine(ep_plan* plan, int32_t layer, const void* d_expert_out, const float* d_weights,
+                       void* d_out, int32_t out_dtype, void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!plan->planned[layer]) return EP_ERR_NOT_PLANNED;
+  if (out_dtype != 0 && out_dtype != 1) return EP_ERR_INVALID_ARGUMENT;
+  if ((int64_t)plan->d.R * plan->d.T > 0 && (!d_expert_out || !d_weights || !d_out))
+    return EP_ERR_INVALID_ARGUMENT;
+  if (!aligned16(d_expert_out) || !aligned16(d_out) ||
+      (reinterpret_cast<uintptr_t>(d_weights) & 3u) != 0)
+    return EP_ERR_INVALID_ARGUMENT;
+  return cuda_status(ep::launch_combine(plan->d, layer_buf(plan, layer), d_expert_out, d_weights,
+                                        d_out, out_dtype, plan->num_sms,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 ep_status_t ep_stage_replicas(ep_plan* plan, int32_t layer, const void* d_native_w,
                               void* d_slots, void* stream) {
   ep_status_t st = check_layer(plan, layer);

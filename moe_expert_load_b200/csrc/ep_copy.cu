@@ -12,6 +12,7 @@
 // every destination with 16-byte vector stores.  See k_permute for the
 // measurements that chose this over bulk-copy (TMA) staging through shared
 // memory.  Nothing here waits on another thread, block or device.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -93,6 +94,118 @@ __global__ void __launch_bounds__(kPermuteThreads) k_permute(PermuteArgs a) {
     }
   }
   if (__any_sync(kFull, overflow) && lane == 0) atomicOr(&a.stats->status, EP_DEV_OUT_CAPACITY);
+}
+
+// ---------------------------------------------------------------------------
+// Combine: the reverse of the dispatch.  One warp per token at a time
+// (grid-stride): lanes 0..K-1 fetch the token's dispatch rows and gate
+// weights, lane K its shared-slot row; the warp walks the hidden dimension in
+// passes of 512 elements (two 16-byte words per lane) and, per pass, loads the
+// rows of four k at a time before their fused multiply-adds, keeping
+// acc = fma(w_k, x_k, acc) in ascending k and adding the shared row last.
+// ---------------------------------------------------------------------------
+struct CombineArgs {
+  const uint4* x;        // [rows][row16] bf16 expert outputs
+  const float* w;        // [N][K]
+  const int32_t* dst_row;
+  const int32_t* shared_row;  // null without a shared expert
+  void* out;             // [N][hidden] bf16 or fp32
+  int64_t N;
+  int row16;
+  int K;
+  int out_f32;
+};
+
+constexpr int kCombineThreads = 256;
+constexpr int kCW = 2;   // 16-byte words per lane per pass
+constexpr int kCK = 4;   // rows whose loads are issued together
+
+__device__ __forceinline__ void fma_bf16x8(float* acc, const uint4 v, float w) {
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = __fmaf_rn(w, __uint_as_float(u[i] << 16), acc[2 * i]);
+    acc[2 * i + 1] = __fmaf_rn(w, __uint_as_float(u[i] & 0xffff0000u), acc[2 * i + 1]);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+__global__ void __launch_bounds__(kCombineThreads) k_combine(CombineArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int row16 = a.row16;
+  for (int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < a.N; n += nw) {
+    int d = -1;
+    float wk = 0.f;
+    if (lane < a.K) {
+      d = a.dst_row[n * a.K + lane];
+      wk = a.w[n * a.K + lane];
+    }
+    const int ds = a.shared_row ? a.shared_row[n] : -1;
+    for (int c0 = 0; c0 < row16; c0 += kCW * 32) {
+      float acc[kCW * 8];
+#pragma unroll
+      for (int i = 0; i < kCW * 8; ++i) acc[i] = 0.f;
+      for (int k0 = 0; k0 < a.K; k0 += kCK) {
+        uint4 v[kCK][kCW];
+        int dk[kCK];
+        float wkk[kCK];
+#pragma unroll
+        for (int j = 0; j < kCK; ++j) {
+          dk[j] = __shfl_sync(kFull, d, (k0 + j) & 31);
+          wkk[j] = __shfl_sync(kFull, wk, (k0 + j) & 31);
+          if (k0 + j >= a.K) dk[j] = -1;
+#pragma unroll
+          for (int c = 0; c < kCW; ++c) {
+            const int idx = c0 + c * 32 + lane;
+            if (dk[j] >= 0 && idx < row16) v[j][c] = a.x[(int64_t)dk[j] * row16 + idx];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kCK; ++j)
+          if (dk[j] >= 0) {
+#pragma unroll
+            for (int c = 0; c < kCW; ++c)
+              if (c0 + c * 32 + lane < row16) fma_bf16x8(acc + c * 8, v[j][c], wkk[j]);
+          }
+      }
+      if (ds >= 0) {
+#pragma unroll
+        for (int c = 0; c < kCW; ++c) {
+          const int idx = c0 + c * 32 + lane;
+          if (idx < row16) {
+            const uint4 v = a.x[(int64_t)ds * row16 + idx];
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[c * 8 + 2 * i] = __fadd_rn(acc[c * 8 + 2 * i], __uint_as_float(u[i] << 16));
+              acc[c * 8 + 2 * i + 1] =
+                  __fadd_rn(acc[c * 8 + 2 * i + 1], __uint_as_float(u[i] & 0xffff0000u));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kCW; ++c) {
+        const int idx = c0 + c * 32 + lane;
+        if (idx >= row16) continue;
+        const float* f = acc + c * 8;
+        if (a.out_f32) {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + (n * row16 + idx) * 8);
+          o[0] = make_float4(f[0], f[1], f[2], f[3]);
+          o[1] = make_float4(f[4], f[5], f[6], f[7]);
+        } else {
+          reinterpret_cast<uint4*>(a.out)[n * row16 + idx] =
+              make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                         pack_bf16x2(f[6], f[7]));
+        }
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -292,6 +405,23 @@ cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden
   // 12 blocks of 4 warps per SM, about twice what is resident at once:
   // measured 6.0 (8), 6.1-6.2 (12) and 6.1 (16) TB/s on the qwen layer
   k_permute<<<(unsigned)(num_sms * 12), kPermuteThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Dims& d, const LayerBuf& L, const void* x, const float* w, void* out,
+                           int out_f32, int num_sms, cudaStream_t st) {
+  CombineArgs a;
+  a.x = static_cast<const uint4*>(x);
+  a.w = w;
+  a.dst_row = L.dst_row;
+  a.shared_row = d.sh ? L.shared_row : nullptr;
+  a.out = out;
+  a.N = (int64_t)d.R * d.T;
+  a.row16 = d.hidden * 2 / 16;
+  a.K = d.K;
+  a.out_f32 = out_f32;
+  if (a.N == 0) return cudaSuccess;
+  k_combine<<<(unsigned)(num_sms * 8), kCombineThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -100,6 +100,8 @@ cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s,
 cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden, void* out,
                             int64_t cap_rows, int rank_begin, int rank_end, int num_sms,
                             cudaStream_t st);
+cudaError_t launch_combine(const Dims& d, const LayerBuf& L, const void* x, const float* w, void* out,
+                           int out_f32, int num_sms, cudaStream_t st);
 cudaError_t launch_stage(const Dims& d, const LayerBuf& L, const void* native_w, void* slots,
                          int num_sms, cudaStream_t st);
 cudaError_t launch_reduce(const Dims& d, const LayerBuf& L, void* slot_grads, int grad_f32,

@@ -222,6 +222,19 @@ def permute_range(p: Plan, hidden_rows: np.ndarray, n0: int, out: np.ndarray) ->
     _load().orc_permute(n, p.K, hidden_rows.strides[0], _p(hidden_rows), _p(dst), _p(srow), _p(out))
 
 
+def combine_tokens(expert_out: np.ndarray, dst_row: np.ndarray, weights: np.ndarray,
+                   shared_row: Optional[np.ndarray] = None) -> np.ndarray:
+    """fp64 combine of selected tokens: dst_row / weights [n][K], shared_row [n]."""
+    x = np.ascontiguousarray(expert_out, dtype=np.uint16)
+    dst = np.ascontiguousarray(dst_row, dtype=np.int64)
+    n, K = dst.shape
+    wt = np.ascontiguousarray(weights, dtype=np.float32).reshape(n, K)
+    srow = None if shared_row is None else np.ascontiguousarray(shared_row, dtype=np.int64).reshape(n)
+    out = np.zeros((n, x.shape[1]), np.float64)
+    _load().orc_combine(n, K, x.shape[1], _p(x), _p(dst), _p(wt), _p(srow), _p(out))
+    return out
+
+
 def combine(p: Plan, expert_out: np.ndarray, weights: np.ndarray) -> np.ndarray:
     """fp64 combine: gate-weighted sum of each token's routed rows, plus its
     shared-expert row with weight 1.  expert_out: bf16 bits (uint16) [rows][H];

@@ -267,3 +267,45 @@ def test_plans_of_different_shapes_coexist():
     dst = pa.view(0)["dst_row"].reshape(wa.N, wa.K).long()
     assert torch.equal(out[dst[:, 0]].view(torch.int16), ha.view(torch.int16))
     assert pa.read_layer_stats(0)["status"] == 0 and pb.read_layer_stats(0)["status"] == 0
+
+
+# ---- combine (reverse of the dispatch) ------------------------------------------
+def _combine_bound(x_bits, dst, w, srow):
+    """sum over terms of |w x| (the scale of the fp32 rounding error)."""
+    ax = (x_bits & 0x7FFF).astype(np.uint16)  # |x| in bf16 bits
+    return oracle.combine_tokens(ax, dst, np.abs(w), srow)
+
+
+@pytest.mark.parametrize("name,shared,out_dtype,sample", [
+    ("tiny", False, "f32", None), ("tiny", True, "f32", None), ("tiny", True, "bf16", None),
+    ("qwen", False, "bf16", 700), ("dsv3", True, "f32", 500)])
+def test_combine_matches_oracle(name, shared, out_dtype, sample):
+    w_cfg = get_config(name).replace(shared_expert=shared)
+    ids = topk_ids(get_config(name))
+    if name == "tiny":
+        ids = ids.copy()
+        ids[2, 5, 1] = -1  # a dropped id contributes nothing
+    plan = gpu_plan(w_cfg, ids)
+    rows = plan.read_layer_stats(0)["rows"]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(21)
+    x = torch.randn((rows, w_cfg.hidden), generator=g, device="cuda").to(torch.bfloat16)
+    wts = torch.rand((w_cfg.R, w_cfg.T, w_cfg.K), generator=g, device="cuda")
+    dt = torch.float32 if out_dtype == "f32" else torch.bfloat16
+    y = plan.combine(0, x, wts, out_dtype=dt)
+    torch.cuda.synchronize()
+    v = plan.view(0)
+    N = w_cfg.N
+    toks = np.arange(N) if sample is None else np.random.default_rng(5).choice(N, sample, replace=False)
+    dst = v["dst_row"].reshape(N, w_cfg.K).cpu().numpy()[toks]
+    srow = None if not shared else v["shared_row"].reshape(N).cpu().numpy()[toks]
+    xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
+    wn = wts.reshape(N, w_cfg.K).cpu().numpy()[toks]
+    want = oracle.combine_tokens(xb, dst, wn, srow)
+    bound = _combine_bound(xb, dst, wn, srow)
+    got = y.float().cpu().numpy()[toks].astype(np.float64)
+    # fp32: K+1 rounded fma/add steps, each within 2^-24 of the running sum
+    tol = 2.0**-20 * bound
+    if out_dtype == "bf16":  # plus one round-to-nearest to 8 significant bits
+        tol = tol + 2.0**-8 * np.abs(want)
+    assert (np.abs(got - want) <= tol + 1e-30).all(), float(np.max(np.abs(got - want) - tol))

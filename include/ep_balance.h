@@ -98,7 +98,9 @@ typedef struct ep_config {
   int32_t num_cap_candidates;       /* J: caps ceil(A(200+j)/(200R)), j < J */
   int32_t shared_expert;            /* 1: one Waterfill shared-expert slot per token ([W]) */
   int32_t waterfill_bonus_permille; /* local preference B = ceil(H*bonus/1000) */
-  int32_t reserved0;                /* must be 0 */
+  int32_t waterfill_all_ranks;      /* 0: candidates = own rank + ranks the token visits
+                                       (communication-conservative set, [W]); 1: all ranks
+                                       ([W]'s all-rank mode) */
   int64_t expert_weight_elems;      /* Wn: bf16 elements of one expert (3*hidden*ffn) */
   uint64_t waterfill_seed;          /* seed of the per-token SplitMix64 draw */
 } ep_config;
@@ -241,12 +243,15 @@ EP_API ep_status_t ep_combine(ep_plan* plan, int32_t layer, const void* d_expert
  * candidates = own rank, then the other ranks the token visits, ascending; draw
  * proportional to slack (+B on the own rank) with u = ((h>>32)*sum)>>32,
  * h = SplitMix64(seed + r*T + t); with no slack, the least-loaded candidate
- * unless the own rank is within B of it.  Writes d_pick [R][T] and d_count [R]
- * (tokens per rank).  Limits: R <= 128, K <= 16, R*T*(K+1) < 2^31.
+ * unless the own rank is within B of it.  flags bit 0 (EP_WATERFILL_ALL_RANKS):
+ * every rank is a candidate ([W]'s all-rank mode), own rank first.  Writes
+ * d_pick [R][T] and d_count [R] (tokens per rank).  Limits: R <= 128, K <= 16,
+ * R*T*(K+1) < 2^31.
  */
+#define EP_WATERFILL_ALL_RANKS 1
 EP_API ep_status_t ep_waterfill(int32_t R, int32_t T, int32_t K, const int32_t* d_load,
                          const int32_t* d_dst_rank, uint64_t seed, int32_t bonus_permille,
-                         int32_t* d_pick, int32_t* d_count, void* stream);
+                         int32_t flags, int32_t* d_pick, int32_t* d_count, void* stream);
 
 /*
  * Load matrix without allocation.  The pages have no counterpart: this exists

@@ -70,7 +70,8 @@ def config_from_workload(w, num_layers: Optional[int] = None, **overrides) -> Ep
         slots_per_rank=w.S, min_replica_quota=w.m, hidden=w.hidden,
         num_layers=num_layers if num_layers is not None else w.layers,
         num_cap_candidates=w.J, shared_expert=int(bool(w.shared_expert)),
-        waterfill_bonus_permille=w.waterfill_bonus_permille, reserved0=0,
+        waterfill_bonus_permille=w.waterfill_bonus_permille,
+        waterfill_all_ranks=int(getattr(w, "waterfill_all_ranks", False)),
         expert_weight_elems=w.expert_elems, waterfill_seed=w.waterfill_seed,
     )
     for k, v in overrides.items():
@@ -212,12 +213,12 @@ def _combine_out(plan, expert_out, out, out_dtype):
 
 
 def ep_waterfill(load: torch.Tensor, dst_rank: torch.Tensor, seed: int, bonus_permille: int = 10,
-                 stream=None):
+                 all_ranks: bool = False, stream=None):
     """Standalone Waterfill: load int32 [R], dst_rank int32 [R][T][K] -> (pick [R][T], count [R])."""
     R, T, K = dst_rank.shape
     pick = torch.empty((R, T), dtype=torch.int32, device=dst_rank.device)
     count = torch.empty((R,), dtype=torch.int32, device=dst_rank.device)
     _check("ep_waterfill", _abi.load().ep_waterfill(
         R, T, K, _ptr(load), _ptr(dst_rank), ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), bonus_permille,
-        _ptr(pick), _ptr(count), _stream(stream)))
+        1 if all_ranks else 0, _ptr(pick), _ptr(count), _stream(stream)))
     return pick, count

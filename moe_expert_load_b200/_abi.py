@@ -38,7 +38,7 @@ class EpConfig(ctypes.Structure):
         ("slots_per_rank", ctypes.c_int32), ("min_replica_quota", ctypes.c_int32),
         ("hidden", ctypes.c_int32), ("num_layers", ctypes.c_int32),
         ("num_cap_candidates", ctypes.c_int32), ("shared_expert", ctypes.c_int32),
-        ("waterfill_bonus_permille", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("waterfill_bonus_permille", ctypes.c_int32), ("waterfill_all_ranks", ctypes.c_int32),
         ("expert_weight_elems", ctypes.c_int64), ("waterfill_seed", ctypes.c_uint64),
     ]
 
@@ -102,7 +102,7 @@ def load():
         "ep_dispatch_layout": (S, [P, I32, P, P, I64, I32, I32, P]),
         "ep_stage_replicas": (S, [P, I32, P, P, P]),
         "ep_reduce_replica_grads": (S, [P, I32, P, I32, P, P]),
-        "ep_waterfill": (S, [I32, I32, I32, P, P, ctypes.c_uint64, I32, P, P, P]),
+        "ep_waterfill": (S, [I32, I32, I32, P, P, ctypes.c_uint64, I32, I32, P, P, P]),
         "ep_combine": (S, [P, I32, P, P, P, I32, P]),
         "ep_status_string": (ctypes.c_char_p, [S]),
         "ep_abi_version": (I32, []),

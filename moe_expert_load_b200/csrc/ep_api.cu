@@ -44,12 +44,12 @@ struct Bump {
 
 ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
   if (!c) return EP_ERR_INVALID_ARGUMENT;
-  if (c->reserved0 != 0) return EP_ERR_INVALID_ARGUMENT;
   const int R = c->num_ranks, E = c->num_experts, K = c->top_k, T = c->tokens_per_rank;
   if (R < 1 || E < 1 || K < 1 || T < 0 || c->slots_per_rank < 0 || c->min_replica_quota < 1 ||
       c->num_layers < 1 || c->num_cap_candidates < 1 || c->hidden < 1 ||
       c->expert_weight_elems < 0 || c->waterfill_bonus_permille < 0 ||
-      (c->shared_expert != 0 && c->shared_expert != 1))
+      (c->shared_expert != 0 && c->shared_expert != 1) ||
+      (c->waterfill_all_ranks != 0 && c->waterfill_all_ranks != 1))
     return EP_ERR_INVALID_ARGUMENT;
   const int Gmax = E / R + (E % R ? 1 : 0);
   if (R > ep::kMaxR || E > ep::kMaxE || Gmax > ep::kMaxNat || K > ep::kMaxK ||
@@ -73,8 +73,8 @@ ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
   d->G = Gmax + d->S + d->sh;
   d->nsub = (T + ep::kSubT - 1) / ep::kSubT;
   d->bonus = c->waterfill_bonus_permille;
+  d->all_ranks = c->waterfill_all_ranks;
   d->hidden = c->hidden;
-  d->pad_ = 0;
   d->seed = c->waterfill_seed;
   d->Wn = c->expert_weight_elems;
   return EP_OK;
@@ -376,14 +376,16 @@ ep_status_t ep_reduce_replica_grads(ep_plan* plan, int32_t layer, void* d_slot_g
 
 ep_status_t ep_waterfill(int32_t R, int32_t T, int32_t K, const int32_t* d_load,
                          const int32_t* d_dst_rank, uint64_t seed, int32_t bonus_permille,
-                         int32_t* d_pick, int32_t* d_count, void* stream) {
-  if (R < 1 || T < 0 || K < 0 || bonus_permille < 0) return EP_ERR_INVALID_ARGUMENT;
+                         int32_t flags, int32_t* d_pick, int32_t* d_count, void* stream) {
+  if (R < 1 || T < 0 || K < 0 || bonus_permille < 0 || (flags & ~EP_WATERFILL_ALL_RANKS) != 0)
+    return EP_ERR_INVALID_ARGUMENT;
   if (R > ep::kMaxR || K > ep::kMaxK || bonus_permille > 1000) return EP_ERR_UNSUPPORTED;
   if ((int64_t)R * T * (K + 1) >= (int64_t)INT32_MAX) return EP_ERR_UNSUPPORTED;
   if (!d_load || !d_count) return EP_ERR_INVALID_ARGUMENT;
   if (T > 0 && (!d_pick || (K > 0 && !d_dst_rank))) return EP_ERR_INVALID_ARGUMENT;
   return cuda_status(ep::launch_waterfill(R, T, K, d_load, d_dst_rank, seed, bonus_permille,
-                                          d_pick, d_count, static_cast<cudaStream_t>(stream)));
+                                          flags & EP_WATERFILL_ALL_RANKS, d_pick, d_count,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -27,7 +27,7 @@ struct Dims {
   int nsub;          // sub-chunks per rank = ceil(T / kSubT)
   int bonus;         // Waterfill local preference, permille
   int hidden;        // bf16 elements per hidden row
-  int pad_;
+  int all_ranks;     // Waterfill candidates: every rank
   uint64_t seed;     // Waterfill draw seed
   int64_t Wn;        // bf16 elements per expert
 };
@@ -107,7 +107,7 @@ cudaError_t launch_stage(const Dims& d, const LayerBuf& L, const void* native_w,
 cudaError_t launch_reduce(const Dims& d, const LayerBuf& L, void* slot_grads, int grad_f32,
                           float* native_grads, int num_sms, cudaStream_t st);
 cudaError_t launch_waterfill(int R, int T, int K, const int32_t* load, const int32_t* dst_rank,
-                             uint64_t seed, int bonus, int32_t* pick, int32_t* count,
+                             uint64_t seed, int bonus, int all_ranks, int32_t* pick, int32_t* count,
                              cudaStream_t st);
 
 }  // namespace ep

@@ -597,6 +597,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   }
 }
 
+// Every rank below R set (all-rank Waterfill candidates).
+__device__ __forceinline__ void mask_all(unsigned (&mask)[kRW], int R) {
+#pragma unroll
+  for (int w = 0; w < kRW; ++w) {
+    const int n = min(max(R - 32 * w, 0), 32);
+    mask[w] = n == 32 ? 0xffffffffu : ((1u << n) - 1u);
+  }
+}
+
 // Set / clear bit q of a 4-word rank mask without a dynamic word index.
 __device__ __forceinline__ void mask_set(unsigned (&mask)[kRW], int q) {
   const unsigned bit = 1u << (q & 31);
@@ -853,9 +862,13 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
       int c = -1;
       if (tt < t1) {
         unsigned mask[kRW] = {0u, 0u, 0u, 0u};
-        for (int k = 0; k < K; ++k) {
-          const int q = dr[(tt - t0) * K + k];
-          if (q != kNoRank) mask_set(mask, q);
+        if (d.all_ranks) {
+          mask_all(mask, R);
+        } else {
+          for (int k = 0; k < K; ++k) {
+            const int q = dr[(tt - t0) * K + k];
+            if (q != kNoRank) mask_set(mask, q);
+          }
         }
         mask_clear(mask, r);
         c = wf_pick(r, (int64_t)r * d.T + tt, mask, s_slack, s_W, B, d.seed);
@@ -975,7 +988,7 @@ __global__ void __launch_bounds__(kScanThreads) k_shared_scan(Dims d, LayerBuf L
 // block from the loads (R <= 128 values).
 __global__ void __launch_bounds__(256)
 k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
-            const int32_t* __restrict__ dst_rank, uint64_t seed, int bonus,
+            const int32_t* __restrict__ dst_rank, uint64_t seed, int bonus, int all_ranks,
             int32_t* __restrict__ pick, int32_t* __restrict__ count) {
   __shared__ int32_t s_load[kMaxR], s_slack[kMaxR];
   __shared__ int64_t s_sum;
@@ -996,9 +1009,13 @@ k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
   if (tok >= N) return;
   const int r = (int)(tok / T);
   unsigned mask[kRW] = {0u, 0u, 0u, 0u};
-  for (int k = 0; k < K; ++k) {
-    const int q = dst_rank[tok * K + k];
-    if (q >= 0 && q < R) mask_set(mask, q);
+  if (all_ranks) {
+    mask_all(mask, R);
+  } else {
+    for (int k = 0; k < K; ++k) {
+      const int q = dst_rank[tok * K + k];
+      if (q >= 0 && q < R) mask_set(mask, q);
+    }
   }
   mask_clear(mask, r);
   const int c = wf_pick(r, tok, mask, s_slack, s_load, B, seed);
@@ -1083,14 +1100,14 @@ cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, c
 }
 
 cudaError_t launch_waterfill(int R, int T, int K, const int32_t* load, const int32_t* dst_rank,
-                             uint64_t seed, int bonus, int32_t* pick, int32_t* count,
+                             uint64_t seed, int bonus, int all_ranks, int32_t* pick, int32_t* count,
                              cudaStream_t st) {
   cudaError_t err = cudaMemsetAsync(count, 0, sizeof(int32_t) * (size_t)R, st);
   if (err != cudaSuccess) return err;
   const int64_t N = (int64_t)R * T;
   if (N > 0)
     k_waterfill<<<(unsigned)((N + 255) / 256), 256, 0, st>>>(R, T, K, load, dst_rank, seed, bonus,
-                                                             pick, count);
+                                                             all_ranks, pick, count);
   return cudaGetLastError();
 }
 

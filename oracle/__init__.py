@@ -33,7 +33,7 @@ class _Cfg(ctypes.Structure):
         ("R", ctypes.c_int32), ("E", ctypes.c_int32), ("K", ctypes.c_int32), ("T", ctypes.c_int32),
         ("S", ctypes.c_int32), ("m", ctypes.c_int32), ("J", ctypes.c_int32),
         ("shared_expert", ctypes.c_int32), ("bonus_permille", ctypes.c_int32),
-        ("pad_", ctypes.c_int32), ("seed", ctypes.c_uint64),
+        ("all_ranks", ctypes.c_int32), ("seed", ctypes.c_uint64),
     ]
 
 
@@ -64,12 +64,15 @@ def _load():
         lib.orc_gmax.restype = ctypes.c_int32
         lib.orc_waterline.argtypes = [ctypes.c_int32, ctypes.c_int64, P, ctypes.c_int32, P, P, P]
         lib.orc_waterline.restype = None
-        lib.orc_waterfill.argtypes = [ctypes.c_int32] * 3 + [P, P, ctypes.c_uint64, ctypes.c_int32, P, P]
+        lib.orc_waterfill.argtypes = [ctypes.c_int32] * 3 + [P, P, ctypes.c_uint64, ctypes.c_int32,
+                                                             ctypes.c_int32, P, P]
         lib.orc_waterfill.restype = ctypes.c_int
         lib.orc_permute.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int64, P, P, P, P]
         lib.orc_permute.restype = None
         lib.orc_combine.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P]
         lib.orc_combine.restype = None
+        lib.orc_eplb_plus.argtypes = [ctypes.c_int32] * 3 + [P, P, P, P]
+        lib.orc_eplb_plus.restype = ctypes.c_int32
         lib.orc_stage.argtypes = [ctypes.c_int32] * 4 + [P, ctypes.c_int64, P, P]
         lib.orc_stage.restype = None
         lib.orc_reduce_grads.argtypes = [ctypes.c_int32] * 4 + [P, ctypes.c_int64, ctypes.c_int32, P, P]
@@ -125,13 +128,14 @@ def gmax(E: int, R: int) -> int:
 
 
 def plan(ids: np.ndarray, *, E: int, S: int, m: int, J: int = 16, shared_expert: bool = False,
-         seed: int = 0, bonus_permille: int = 10) -> Plan:
+         seed: int = 0, bonus_permille: int = 10, all_ranks: bool = False) -> Plan:
     """Whole balance + dispatch plan of one layer from gate ids [R][T][K]."""
     lib = _load()
     ids = np.ascontiguousarray(ids, dtype=np.int32)
     R, T, K = ids.shape
     cfg = _Cfg(R=R, E=E, K=K, T=T, S=S, m=m, J=J, shared_expert=int(bool(shared_expert)),
-               bonus_permille=bonus_permille, pad_=0, seed=seed & 0xFFFFFFFFFFFFFFFF)
+               bonus_permille=bonus_permille, all_ranks=int(bool(all_ranks)),
+               seed=seed & 0xFFFFFFFFFFFFFFFF)
     Gm = gmax(E, R)
     G = Gm + S + (1 if shared_expert else 0)
     L = np.zeros((R, E), np.int64)
@@ -186,7 +190,8 @@ def waterline(load: np.ndarray, N: int, bonus_permille: int = 10):
     return int(H.value), int(B.value), slack
 
 
-def waterfill(load: np.ndarray, dst_rank: np.ndarray, *, seed: int, bonus_permille: int = 10):
+def waterfill(load: np.ndarray, dst_rank: np.ndarray, *, seed: int, bonus_permille: int = 10,
+              all_ranks: bool = False):
     """Standalone Waterfill: shared-slot rank per token and per-rank counts."""
     load = np.ascontiguousarray(load, dtype=np.int64)
     dst_rank = np.ascontiguousarray(dst_rank, dtype=np.int32)
@@ -194,7 +199,7 @@ def waterfill(load: np.ndarray, dst_rank: np.ndarray, *, seed: int, bonus_permil
     pick = np.zeros((R, T), np.int32)
     count = np.zeros(R, np.int64)
     rc = _load().orc_waterfill(R, T, K, _p(load), _p(dst_rank), seed & 0xFFFFFFFFFFFFFFFF,
-                               bonus_permille, _p(pick), _p(count))
+                               bonus_permille, int(bool(all_ranks)), _p(pick), _p(count))
     if rc != 0:
         raise ValueError("oracle waterfill rejected its arguments")
     return pick, count
@@ -220,6 +225,18 @@ def permute_range(p: Plan, hidden_rows: np.ndarray, n0: int, out: np.ndarray) ->
     dst = np.ascontiguousarray(p.dst_row.reshape(-1, p.K)[n0:n0 + n])
     srow = None if p.shared_row is None else np.ascontiguousarray(p.shared_row.reshape(-1)[n0:n0 + n])
     _load().orc_permute(n, p.K, hidden_rows.strides[0], _p(hidden_rows), _p(dst), _p(srow), _p(out))
+
+
+def eplb_plus(Tot: np.ndarray, R: int, S: int):
+    """EPLB+ comparison baseline: (inst_expert [R][G], inst_quota [R][G], W [R], replicas)."""
+    Tot = np.ascontiguousarray(Tot, dtype=np.int64)
+    E = Tot.shape[0]
+    G = gmax(E, R) + S
+    ie = np.zeros((R, G), np.int32)
+    iq = np.zeros((R, G), np.int64)
+    W = np.zeros(R, np.int64)
+    n = _load().orc_eplb_plus(R, E, S, _p(Tot), _p(ie), _p(iq), _p(W))
+    return ie, iq, W, int(n)
 
 
 def combine_tokens(expert_out: np.ndarray, dst_row: np.ndarray, weights: np.ndarray,

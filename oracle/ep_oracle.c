@@ -60,7 +60,7 @@ typedef struct {
   int32_t J;              /* number of cap candidates */
   int32_t shared_expert;  /* 1: one Waterfill shared-expert slot per token */
   int32_t bonus_permille; /* local preference of the Waterfill draw */
-  int32_t pad_;
+  int32_t all_ranks;      /* 1: Waterfill candidates are all ranks, not only visited ones */
   uint64_t seed;          /* Waterfill draw seed */
 } orc_cfg;
 
@@ -157,11 +157,17 @@ static int32_t waterfill_pick(const int32_t* cand, int32_t nc, const int64_t* lo
   return (load[cand[0]] <= load[lo] + B) ? cand[0] : lo;
 }
 
-/* candidate list of a token: own rank, then distinct other ranks ascending */
+/* candidate list of a token: own rank, then the distinct other ranks it
+ * visits ascending — or, in all-rank mode, every other rank ascending */
 static int32_t waterfill_candidates(int32_t r, const int32_t* ranks, int32_t K, int32_t R,
-                                    int32_t* cand) {
+                                    int32_t all_ranks, int32_t* cand) {
   int32_t nc = 0;
   cand[nc++] = r;
+  if (all_ranks) {
+    for (int32_t q = 0; q < R; ++q)
+      if (q != r) cand[nc++] = q;
+    return nc;
+  }
   for (int32_t k = 0; k < K; ++k) {
     const int32_t q = ranks[k];
     if (q < 0 || q >= R) continue;
@@ -477,7 +483,7 @@ int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int
     int64_t H, B;
     int64_t* slack = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
     orc_waterline(R, (int64_t)R * T, W, c->bonus_permille, &H, &B, slack);
-    int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K + 1));
+    int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K + R + 1));
     int32_t* ranks = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
     for (int32_t r = 0; r < R; ++r)
       for (int32_t t = 0; t < T; ++t) {
@@ -485,7 +491,7 @@ int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int
           const int32_t i = dst_inst[((int64_t)r * T + t) * K + k];
           ranks[k] = i < 0 ? -1 : i / G;
         }
-        const int32_t nc = waterfill_candidates(r, ranks, K, R, cand);
+        const int32_t nc = waterfill_candidates(r, ranks, K, R, c->all_ranks, cand);
         const int32_t pick = waterfill_pick(cand, nc, W, slack, B, c->seed, (int64_t)r * T + t);
         shared_rank[(int64_t)r * T + t] = pick;
         shared_cnt[pick] += 1;
@@ -541,15 +547,17 @@ int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int
 /* load[R]: routed load per rank; dst_rank[R][T][K]: destination rank of each
  * routed assignment (-1 = none).  Writes pick[R][T] and count[R]. */
 int orc_waterfill(int32_t R, int32_t T, int32_t K, const int64_t* load, const int32_t* dst_rank,
-                  uint64_t seed, int32_t bonus_permille, int32_t* pick_out, int64_t* count) {
+                  uint64_t seed, int32_t bonus_permille, int32_t all_ranks, int32_t* pick_out,
+                  int64_t* count) {
   int64_t H, B;
   int64_t* slack = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
-  int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K + 1));
+  int32_t* cand = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K + R + 1));
   orc_waterline(R, (int64_t)R * T, load, bonus_permille, &H, &B, slack);
   for (int32_t q = 0; q < R; ++q) count[q] = 0;
   for (int32_t r = 0; r < R; ++r)
     for (int32_t t = 0; t < T; ++t) {
-      const int32_t nc = waterfill_candidates(r, dst_rank + ((int64_t)r * T + t) * K, K, R, cand);
+      const int32_t nc =
+          waterfill_candidates(r, dst_rank + ((int64_t)r * T + t) * K, K, R, all_ranks, cand);
       const int32_t pick = waterfill_pick(cand, nc, load, slack, B, seed, (int64_t)r * T + t);
       pick_out[(int64_t)r * T + t] = pick;
       count[pick] += 1;
@@ -569,6 +577,85 @@ void orc_permute(int64_t N, int32_t K, int64_t row_bytes, const uint8_t* hidden,
     }
     if (shared_row) memcpy(out + shared_row[n] * row_bytes, hidden + n * row_bytes, (size_t)row_bytes);
   }
+}
+
+/* ---- EPLB+ comparison baseline ------------------------------------------ */
+/* UltraEP page, section "Quota decides replicas and token split together":
+ * EPLB+ uses the same exact per-layer loads but EPLB-style replication and
+ * round-robin rerouting.  Reading (the page does not spell EPLB out): every
+ * redundant slot is filled, one at a time, with a replica of the expert whose
+ * load per instance T[e]/n[e] is largest (smallest e on ties) among experts
+ * that still fit somewhere, placed on the rank with the smallest estimated
+ * load sum_i T[e_i]/n[e_i] that has a free slot and no instance of the expert
+ * (smallest rank on ties); then each expert's tokens are split round robin
+ * over its instances in instance order (the first T[e] mod n instances get one
+ * more).  Writes the instance table like orc_plan and W[R]; returns the number
+ * of replicas placed. */
+int32_t orc_eplb_plus(int32_t R, int32_t E, int32_t S, const int64_t* Tot, int32_t* inst_expert,
+                      int64_t* inst_quota, int64_t* W) {
+  const int32_t Gmax = orc_gmax(E, R), G = Gmax + S;
+  int32_t* n = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+  int32_t* used = (int32_t*)calloc((size_t)R, sizeof(int32_t));
+  double* est = (double*)calloc((size_t)R, sizeof(double));
+  for (int32_t e = 0; e < E; ++e) n[e] = 1;
+  for (int32_t q = 0; q < R; ++q)
+    for (int32_t col = 0; col < G; ++col) {
+      inst_expert[(int64_t)q * G + col] = -1;
+      inst_quota[(int64_t)q * G + col] = 0;
+    }
+  for (int32_t q = 0; q < R; ++q)
+    for (int32_t i = 0; i < nat_count(q, E, R); ++i)
+      inst_expert[(int64_t)q * G + i] = nat_first(q, E, R) + i;
+  int32_t placed = 0;
+  for (int32_t round = 0; round < R * S; ++round) {
+    /* estimated load of each rank with the current instance counts */
+    for (int32_t q = 0; q < R; ++q) {
+      est[q] = 0.0;
+      for (int32_t col = 0; col < G; ++col) {
+        const int32_t e = inst_expert[(int64_t)q * G + col];
+        if (e >= 0) est[q] += (double)Tot[e] / n[e];
+      }
+    }
+    int32_t best_e = -1, best_r = -1;
+    for (int32_t e = 0; e < E; ++e) {
+      /* candidate only if some rank has a free slot and no instance of e */
+      int32_t r_for_e = -1;
+      for (int32_t q = 0; q < R; ++q) {
+        if (used[q] >= S) continue;
+        int holds_e = 0;
+        for (int32_t col = 0; col < G; ++col) holds_e |= inst_expert[(int64_t)q * G + col] == e;
+        if (holds_e) continue;
+        if (r_for_e < 0 || est[q] < est[r_for_e]) r_for_e = q;
+      }
+      if (r_for_e < 0) continue;
+      /* largest T[e]/n[e]: compare T[e]*n[b] > T[b]*n[e] exactly */
+      if (best_e < 0 || Tot[e] * n[best_e] > Tot[best_e] * n[e]) {
+        best_e = e;
+        best_r = r_for_e;
+      }
+    }
+    if (best_e < 0) break;
+    inst_expert[(int64_t)best_r * G + Gmax + used[best_r]] = best_e;
+    used[best_r] += 1;
+    n[best_e] += 1;
+    ++placed;
+  }
+  /* round robin over the instances of each expert, in instance order */
+  int32_t* seen = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+  for (int32_t q = 0; q < R; ++q) W[q] = 0;
+  for (int64_t i = 0; i < (int64_t)R * G; ++i) {
+    const int32_t e = inst_expert[i];
+    if (e < 0) continue;
+    const int64_t quota = Tot[e] / n[e] + (seen[e] < Tot[e] % n[e] ? 1 : 0);
+    seen[e] += 1;
+    inst_quota[i] = quota;
+    W[i / G] += quota;
+  }
+  free(seen);
+  free(n);
+  free(used);
+  free(est);
+  return placed;
 }
 
 /* ---- combine (reverse of the dispatch, with gate weights) -------------- */

@@ -11,7 +11,8 @@ from moe_expert_load_b200 import Plan, config_from_workload
 
 def oracle_plan(w, ids, **kw):
     args = dict(E=w.E, S=w.S, m=w.m, J=w.J, shared_expert=w.shared_expert,
-                seed=w.waterfill_seed, bonus_permille=w.waterfill_bonus_permille)
+                seed=w.waterfill_seed, bonus_permille=w.waterfill_bonus_permille,
+                all_ranks=w.waterfill_all_ranks)
     args.update(kw)
     return oracle.plan(ids, **args)
 

@@ -15,7 +15,7 @@ page (section "Waterfill") require of any valid plan:
   corner rule: no two flows cross), and rows inside an instance follow the
   source order;
 * the Waterfill shared slot of a token is on its own rank or on a rank the token
-  already visits.
+  already visits (any rank in all-rank mode).
 """
 from __future__ import annotations
 
@@ -31,7 +31,7 @@ def native_blocks(E: int, R: int):
 
 def check_plan(ids: np.ndarray, E: int, S: int, m: int, *, Gmax: int, G: int, W, inst_expert,
                inst_quota, inst_off, dst_row, cap=None, stop=None, shared_rank=None,
-               shared_row=None, W0=None):
+               shared_row=None, W0=None, all_ranks=False):
     ids = np.asarray(ids)
     R, T, K = ids.shape
     inst_expert = np.asarray(inst_expert).reshape(R, G)
@@ -144,7 +144,10 @@ def check_plan(ids: np.ndarray, E: int, S: int, m: int, *, Gmax: int, G: int, W,
         rank_k[valid] = rank_of_inst
         own = sr == np.arange(R)[:, None]
         visits = (rank_k == sr[:, :, None]).any(axis=2)
-        assert (own | visits).all(), "shared slot outside the candidate set"
+        if all_ranks:
+            assert ((sr >= 0) & (sr < R)).all()
+        else:
+            assert (own | visits).all(), "shared slot outside the candidate set"
         counts = np.bincount(sr.ravel(), minlength=R)
         assert (inst_quota[:, Gmax + S] == counts).all()
         # shared rows ordered by (source rank, t) inside each rank's shared column

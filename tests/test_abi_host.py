@@ -70,7 +70,7 @@ def test_workspace_sizes(name):
 @pytest.mark.parametrize("field,value,code", [
     ("num_ranks", 129, 2), ("num_ranks", 0, 1), ("num_experts", 1025, 2), ("top_k", 17, 2),
     ("slots_per_rank", 9, 2), ("num_cap_candidates", 17, 2), ("hidden", 12, 2),
-    ("expert_weight_elems", 12, 2), ("min_replica_quota", 0, 1), ("reserved0", 1, 1),
+    ("expert_weight_elems", 12, 2), ("min_replica_quota", 0, 1), ("waterfill_all_ranks", 2, 1),
     ("waterfill_bonus_permille", 1001, 2), ("shared_expert", 2, 1), ("tokens_per_rank", -1, 1),
 ])
 def test_config_validation(field, value, code):

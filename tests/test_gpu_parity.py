@@ -219,18 +219,27 @@ def test_reduce_grads_bit_exact(grad_dtype):
 
 
 # ---- standalone Waterfill -------------------------------------------------------
-def test_waterfill_standalone_parity():
+@pytest.mark.parametrize("all_ranks", [False, True])
+def test_waterfill_standalone_parity(all_ranks):
     rng = np.random.default_rng(77)
-    for R, T, K in [(4, 1000, 2), (64, 4096, 8), (7, 333, 5), (128, 50, 16)]:
+    for R, T, K in [(4, 1000, 2), (64, 4096, 8), (7, 333, 5), (128, 50, 16), (33, 100, 0)]:
         load = rng.integers(0, 5 * T, size=R).astype(np.int32)
-        dst = rng.integers(-1, R, size=(R, T, K)).astype(np.int32)
+        dst = rng.integers(-1, R, size=(R, T, max(K, 1))).astype(np.int32)[:, :, :K].copy()
         for seed, bonus in [(1, 10), (2**63 + 5, 0), (99, 500)]:
             pick, count = ep_waterfill(torch.from_numpy(load).cuda(), torch.from_numpy(dst).cuda(),
-                                       seed=seed, bonus_permille=bonus)
+                                       seed=seed, bonus_permille=bonus, all_ranks=all_ranks)
             torch.cuda.synchronize()
-            wp, wc = oracle.waterfill(load, dst, seed=seed, bonus_permille=bonus)
+            wp, wc = oracle.waterfill(load, dst, seed=seed, bonus_permille=bonus, all_ranks=all_ranks)
             np.testing.assert_array_equal(pick.cpu().numpy(), wp)
             np.testing.assert_array_equal(count.cpu().numpy(), wc)
+
+
+def test_plan_parity_waterfill_all_ranks():
+    for name in ("dsv3", "tiny"):
+        w = get_config(name).replace(shared_expert=True, waterfill_all_ranks=True)
+        ids = topk_ids(get_config(name))
+        o = oracle_plan(w, ids)
+        compare_plan(fetch(gpu_plan(w, ids)), o, w)
 
 
 # ---- errors are reported, not trapped --------------------------------------------

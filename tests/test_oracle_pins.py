@@ -493,3 +493,100 @@ def test_combine_is_linear_and_skips_dropped_rows():
     wi = np.ones_like(w)
     np.testing.assert_array_equal(oracle.combine(p, xij, wi), oracle.combine(p, xi, wi) + oracle.combine(p, xj, wi))
     assert yb.shape == ya.shape
+
+
+# ---- Waterfill all-rank mode ----------------------------------------------------
+def test_waterfill_all_ranks_single_slack_rank():
+    # only rank 3 has slack and there is no local bonus: in all-rank mode every
+    # token picks it, whatever ranks it visits (conservative mode would not)
+    R, T, K = 4, 50, 2
+    dst = _dst_ranks(R, T, K, np.random.default_rng(3))
+    load = np.array([500, 500, 500, 0])
+    pick, cnt = oracle.waterfill(load, dst, seed=11, bonus_permille=0, all_ranks=True)
+    assert (pick == 3).all() and cnt.tolist() == [0, 0, 0, R * T]
+    pick_c, _ = oracle.waterfill(load, dst, seed=11, bonus_permille=0, all_ranks=False)
+    assert (pick_c != 3).any()
+
+
+def test_waterfill_all_ranks_proportional():
+    # uniform-slack ranks except rank 0 (no slack): picks spread over ranks 1..3
+    # in proportion to slack, within a 5-sigma binomial bound per rank
+    R, T = 4, 30000
+    load = np.array([5 * T, 0, T // 2, T])
+    H, B, slack = oracle.waterline(load, R * T, 0)
+    dst = np.full((R, T, 1), -1, np.int32)
+    pick, _ = oracle.waterfill(load, dst, seed=4, bonus_permille=0, all_ranks=True)
+    p = slack / slack.sum()
+    n = R * T
+    for q in range(R):
+        f = float((pick == q).mean())
+        assert abs(f - p[q]) <= 5 * np.sqrt(max(p[q] * (1 - p[q]), 1e-12) / n) + 1e-12
+    assert p[0] == 0 and (pick == 0).sum() == 0
+
+
+def test_waterfill_all_ranks_flattens_more():
+    # more freedom than the conservative set: the worst rank (routed + shared)
+    # is no higher, and the spread is tighter, on the dsv3 layer without slots
+    cfg = get_config("dsv3")
+    ids = topk_ids(cfg)
+    pc = _plan_cfg(cfg, ids, S=0)
+    pa = _plan_cfg(cfg, ids, S=0, all_ranks=True)
+    tc = pc.W + pc.inst_quota[:, -1]
+    ta = pa.W + pa.inst_quota[:, -1]
+    assert ta.max() <= tc.max() and ta.std() < tc.std()
+    check_plan(ids, cfg.E, 0, cfg.m, Gmax=pa.Gmax, G=pa.G, W=pa.W, inst_expert=pa.inst_expert,
+               inst_quota=pa.inst_quota, inst_off=pa.inst_off, dst_row=pa.dst_row, cap=pa.cap,
+               stop=pa.stop_name, shared_rank=pa.shared_rank, shared_row=pa.shared_row,
+               all_ranks=True)
+
+
+# ---- EPLB+ comparison baseline and LP cross-check ------------------------------
+def test_eplb_plus_worked_example():
+    g = _golden("quota_worked_examples.json")["eplb_plus_fig_ep4"]
+    ie, iq, W, n = oracle.eplb_plus(np.array(g["Tot"]), g["R"], g["S"])
+    assert ie.tolist() == g["inst_expert"] and iq.tolist() == g["inst_quota"]
+    assert W.tolist() == g["W"] and n == g["replicas"]
+
+
+@pytest.mark.parametrize("name", ["qwen", "dsv3"])
+def test_eplb_plus_is_a_valid_round_robin_plan(name):
+    cfg = get_config(name)
+    p = _plan_cfg(cfg, topk_ids(cfg))
+    ie, iq, W, n = oracle.eplb_plus(p.Tot, cfg.R, cfg.S)
+    Gm = p.Gmax
+    assert n == cfg.R * cfg.S  # EPLB-style: every redundant slot is used
+    per_e = {}
+    for q in range(cfg.R):
+        held = [int(e) for e in ie[q] if e >= 0]
+        assert len(held) == len(set(held))
+        assert (ie[q, Gm:] >= 0).sum() <= cfg.S
+        assert W[q] == iq[q].sum()
+        for col in range(ie.shape[1]):
+            if ie[q, col] >= 0:
+                per_e.setdefault(int(ie[q, col]), []).append(int(iq[q, col]))
+    for e, qs in per_e.items():
+        assert sum(qs) == p.Tot[e]
+        assert max(qs) - min(qs) <= 1 and qs == sorted(qs, reverse=True)  # round robin
+
+
+def test_lp_bound_is_met_on_the_worked_case():
+    from oracle.lplb import min_max_split
+
+    case = _golden("quota_worked_examples.json")["cases"][0]
+    ids = np.array(case["ids"], dtype=np.int32).reshape(case["R"], case["T"], case["K"])
+    p = oracle.plan(ids, E=case["E"], S=case["S"], m=case["m"], J=case["J"])
+    M, x = min_max_split(p.Tot, p.inst_expert, p.Gmax, p.S, m_replica=case["m"])
+    assert abs(M - 9.0) < 1e-9 and p.after_max == 9
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen", "dsv3"])
+def test_greedy_split_is_never_below_the_lp_bound(name):
+    # for the greedy's own placement, no split (LP relaxation, replicas >= m)
+    # has a smaller worst rank; the greedy's split is feasible for that LP
+    from oracle.lplb import min_max_split
+
+    cfg = get_config(name)
+    p = _plan_cfg(cfg, topk_ids(cfg))
+    M, _ = min_max_split(p.Tot, p.inst_expert, p.Gmax, p.S, m_replica=cfg.m)
+    assert p.after_max >= M - 1e-6
+    assert p.after_max <= 1.06 * M  # and close to it on these workloads

@@ -31,6 +31,7 @@ class WorkloadConfig:
     J: int = 16  # cap candidates of the quota solve
     waterfill_seed: int = 0x5EED_0F_1A7E12
     waterfill_bonus_permille: int = 10
+    waterfill_all_ranks: bool = False  # Waterfill candidates: all ranks instead of visited ones
 
     @property
     def N(self) -> int:

@@ -27,7 +27,7 @@ struct Layout {
       shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, stats, tickets;
   size_t layer_bytes;
   // scratch (absolute)
-  size_t sub_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase,
+  size_t sub_cnt, blk_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase,
       shared_tot;
   size_t scratch_bytes;
   size_t total;
@@ -71,7 +71,7 @@ ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
   d->Gmax = Gmax;
   d->sh = c->shared_expert;
   d->G = Gmax + d->S + d->sh;
-  d->nsub = (T + ep::kSubT - 1) / ep::kSubT;
+  d->nsub = (T + ep::kPlanSubT - 1) / ep::kPlanSubT;
   d->bonus = c->waterfill_bonus_permille;
   d->all_ranks = c->waterfill_all_ranks;
   d->hidden = c->hidden;
@@ -107,6 +107,7 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   Bump s;
   s.off = L.layer_bytes * (size_t)num_layers;
   L.sub_cnt = s.take(i4 * (size_t)d.R * d.nsub * d.E);
+  L.blk_cnt = s.take(i4 * (size_t)d.R * ((d.nsub + ep::kPlanWarps - 1) / ep::kPlanWarps) * d.E);
   L.wsub_cnt = s.take(d.sh ? i4 * (size_t)d.R * d.R * d.nsub : 0);
   L.seg_ptr = s.take(i4 * (size_t)d.E * (d.R + 1));
   L.seg_ord = s.take(i4 * (size_t)d.E * 3 * d.R);
@@ -170,6 +171,7 @@ ep::Scratch scratch(const ep_plan* p) {
   const Layout& l = p->lay;
   ep::Scratch s;
   s.sub_cnt = at(p, l.sub_cnt);
+  s.blk_cnt = at(p, l.blk_cnt);
   s.wsub_cnt = p->d.sh ? at(p, l.wsub_cnt) : nullptr;
   s.seg_ptr = at(p, l.seg_ptr);
   s.seg_ord = at(p, l.seg_ord);

@@ -9,7 +9,9 @@
 
 namespace ep {
 
-constexpr int kSubT = 128;      // tokens per sub-chunk; one warp owns one sub-chunk
+constexpr int kSubT = 128;      // tokens per sub-chunk of the static load-matrix variant
+constexpr int kPlanSubT = 64;   // tokens per sub-chunk of the plan kernels (one warp each)
+constexpr int kPlanWarps = 8;   // sub-chunks (warps) per block of the plan kernels
 constexpr int kMaxR = 128;      // ranks (4 words of 32 per warp lane)
 constexpr int kRW = 4;          // rank words per lane: lane owns ranks lane + 32*k
 constexpr int kMaxE = 1024;
@@ -24,7 +26,7 @@ struct Dims {
   int R, E, K, T;
   int S, m, J;
   int Gmax, G, sh;   // natives per rank (max), columns per rank, shared column present
-  int nsub;          // sub-chunks per rank = ceil(T / kSubT)
+  int nsub;          // sub-chunks per rank = ceil(T / kPlanSubT)
   int bonus;         // Waterfill local preference, permille
   int hidden;        // bf16 elements per hidden row
   int all_ranks;     // Waterfill candidates: every rank
@@ -56,7 +58,8 @@ struct LayerBuf {
 
 // Scratch shared by all layers, reused by every balance call.
 struct Scratch {
-  int32_t* sub_cnt;   // [R][nsub][E] per-sub-chunk counts, then exclusive bases
+  int32_t* sub_cnt;   // [R][nsub][E] per-sub-chunk counts
+  int32_t* blk_cnt;   // [R][ceil(nsub/kPlanWarps)][E] per-block counts
   int32_t* wsub_cnt;  // [R][R*nsub] shared-slot counts per (dest rank, sub-chunk), then bases
   int32_t* seg_ptr;   // [E][R+1] first segment of each source rank, per expert
   int32_t* seg_ord;   // [E][3R] first ordinal of the segment

@@ -19,7 +19,7 @@ namespace ep {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kWarpsPerBlock = 8;
+constexpr int kWarpsPerBlock = kPlanWarps;
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -44,35 +44,38 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-constexpr int kBatch = 16;  // ids per lane in flight
+constexpr int kBatch = 16;     // ids per lane in flight in k_hist (a whole sub-chunk for K <= 8)
+constexpr int kAsgBatch = 8;   // ids per lane per pass in k_assign
 
 // ---------------------------------------------------------------------------
-// a1: load histogram.  A block owns up to 8 consecutive sub-chunks of kSubT
-// tokens of one source rank, one per warp.  Each warp counts its sub-chunk into
-// a private shared-memory histogram with shared atomic adds (16 ids per lane in
-// flight, no dependence between rounds); the warp writes its row of counts (the
-// bases of the stable ordinals, used by k_assign), and the block adds the sum
-// of its rows to the load matrix L[r][e] and the expert totals with integer
-// atomics (order-independent, so the result is deterministic).
+// a1: load histogram.  A block owns up to 8 consecutive sub-chunks of
+// kPlanSubT tokens of one source rank, one per warp.  Each warp loads its whole
+// sub-chunk at once (at most 16 ids per lane) and counts it into a private
+// shared-memory histogram with shared atomic adds; the warp writes its row of
+// counts and the block writes the sum of its rows (the two levels of bases of
+// the stable ordinals, used by k_assign).  After the predecessor (the kernel
+// that clears the layer's counters) has finished, the block adds its sum to the
+// load matrix L[r][e] and the expert totals with integer atomics
+// (order-independent, so the result is deterministic).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 6)
 k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, LayerBuf L) {
   extern __shared__ int32_t sm_hist[];
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nbpr = (d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock;
-  const int r = blockIdx.x / nbpr;
-  const int sub = (blockIdx.x - r * nbpr) * kWarpsPerBlock + warp;
+  const int r = blockIdx.x / nbpr, b = blockIdx.x - r * nbpr;
+  const int sub = b * kWarpsPerBlock + warp;
   const int E = d.E, K = d.K;
   int32_t* hist = sm_hist + warp * E;
   for (int e = lane; e < E; e += 32) hist[e] = 0;
   __syncwarp();
   int bad = 0;
   if (sub < d.nsub) {
-    const int t0 = sub * kSubT, t1 = min(d.T, t0 + kSubT);
+    const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
     const int32_t* src = ids + (int64_t)r * d.T * K;
     const int a1 = t1 * K;
-    for (int a = t0 * K; a < a1; a += kBatch * 32) {
+    for (int a = t0 * K; a < a1; a += kBatch * 32) {  // one pass for K <= 16
       int v[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
@@ -88,17 +91,38 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, LayerBuf L) {
     int32_t* out = s.sub_cnt + ((int64_t)r * d.nsub + sub) * E;
     for (int e = lane; e < E; e += 32) out[e] = hist[e];
   }
-  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&L.stats->status, EP_DEV_BAD_ID);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int c = 0;
+  int32_t* blk = s.blk_cnt + ((int64_t)r * nbpr + b) * E;
+  int csum[4];
 #pragma unroll
-    for (int w = 0; w < kWarpsPerBlock; ++w) c += sm_hist[w * E + e];
-    if (c) {
-      atomicAdd(&L.load[r * E + e], c);
-      atomicAdd(&L.expert_total[e], c);
+  for (int u = 0; u < 4; ++u) {
+    const int e = threadIdx.x + u * blockDim.x;
+    csum[u] = 0;
+    if (e < E) {
+#pragma unroll
+      for (int w = 0; w < kWarpsPerBlock; ++w) csum[u] += sm_hist[w * E + e];
+      blk[e] = csum[u];
     }
   }
+  pdl_wait();  // the layer's counters and status word have been cleared
+  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&L.stats->status, EP_DEV_BAD_ID);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int e = threadIdx.x + u * blockDim.x;
+    if (e < E && csum[u]) {
+      atomicAdd(&L.load[r * E + e], csum[u]);
+      atomicAdd(&L.expert_total[e], csum[u]);
+    }
+  }
+}
+
+// Clears the layer's stats, load matrix, expert totals and arrival tickets
+// (adjacent in the layer block) before the histogram adds into them.
+__global__ void __launch_bounds__(256) k_clear_layer(int4* __restrict__ p, int64_t n16) {
+  pdl_trigger();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
+       i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = make_int4(0, 0, 0, 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -109,10 +133,11 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, LayerBuf L) {
 // those with quota >= m — to a new replica on the rank r with the largest slack
 // C - W_r >= m among ranks with a free slot and no instance of e (smallest index
 // on ties).  If no native of p can move, p is stuck.  The run with the smallest
-// (max load, replicas, j) wins.  A lane owns ranks lane + 32k and keeps their
-// load, slot table and flags in registers; native quotas live in shared memory.
+// (max load, replicas, j) wins.  A lane owns ranks lane + 32k (k < RW, the
+// number of 32-rank words) and keeps their load, slot table and flags in
+// registers; native quotas live in shared memory.
 // ---------------------------------------------------------------------------
-template <int SMAX>
+template <int SMAX, int RW>
 __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scratch s) {
   extern __shared__ int32_t sm[];
   int32_t* Tot = sm;              // [E]
@@ -157,14 +182,14 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   const int j = warp;
   const int64_t den = 200LL * R;
   const int C = (int)(((int64_t)A * (200 + j) + den - 1) / den);
-  int Wr[kRW], used[kRW], se[kRW][SMAX], sq[kRW][SMAX];
+  int Wr[RW], used[RW], se[RW][SMAX], sq[RW][SMAX];
   int replicas = 0, stop = -1, maxW = 0;
   if (solver) {
     int32_t* Qn = Qn_all + j * E;
     for (int e = lane; e < E; e += 32) Qn[e] = Tot[e];
     unsigned stuck = 0, slotlim = 0;
 #pragma unroll
-    for (int k = 0; k < kRW; ++k) {
+    for (int k = 0; k < RW; ++k) {
       const int q = lane + 32 * k;
       Wr[k] = q < R ? s_W0[q] : 0;
       used[k] = 0;
@@ -177,13 +202,13 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       if (it >= iter_cap) { stop = EP_STOP_ITER_CAP; break; }
       unsigned lm = 0;
 #pragma unroll
-      for (int k = 0; k < kRW; ++k)
+      for (int k = 0; k < RW; ++k)
         if (lane + 32 * k < R && !((stuck >> k) & 1u)) lm = max(lm, (unsigned)Wr[k]);
       const int vmax = (int)__reduce_max_sync(kFull, lm);
       if (vmax <= C) break;
       int p = -1;
 #pragma unroll
-      for (int k = 0; k < kRW; ++k) {
+      for (int k = 0; k < RW; ++k) {
         const unsigned b = __ballot_sync(
             kFull, lane + 32 * k < R && !((stuck >> k) & 1u) && Wr[k] == vmax);
         if (p < 0 && b) p = 32 * k + __ffs(b) - 1;
@@ -200,9 +225,9 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
         const int e = nf + li;
         // receivers: free slot, no instance of e, slack >= m
         unsigned ls = 0;
-        bool ok[kRW];
+        bool ok[RW];
 #pragma unroll
-        for (int k = 0; k < kRW; ++k) {
+        for (int k = 0; k < RW; ++k) {
           const int q = lane + 32 * k;
           bool h = false;
 #pragma unroll
@@ -217,13 +242,13 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
         }
         int rr = -1;
 #pragma unroll
-        for (int k = 0; k < kRW; ++k) {
+        for (int k = 0; k < RW; ++k) {
           const unsigned b = __ballot_sync(kFull, ok[k] && (unsigned)(C - Wr[k]) == smax);
           if (rr < 0 && b) rr = 32 * k + __ffs(b) - 1;
         }
         const int x = min(min(max(ex, m), (int)smax), (int)qmax);
 #pragma unroll
-        for (int k = 0; k < kRW; ++k) {
+        for (int k = 0; k < RW; ++k) {
           const int q = lane + 32 * k;
           if (q == p) Wr[k] -= x;
           if (q == rr) {
@@ -245,12 +270,12 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       if (!moved) {
         bool fr = false;
 #pragma unroll
-        for (int k = 0; k < kRW; ++k)
+        for (int k = 0; k < RW; ++k)
           fr |= (lane + 32 * k < R && used[k] == S && C - Wr[k] >= m);
         const bool full_receiver = __any_sync(kFull, fr);
         const bool native_big = __any_sync(kFull, lane < nc && myQ >= m);
 #pragma unroll
-        for (int k = 0; k < kRW; ++k)
+        for (int k = 0; k < RW; ++k)
           if (lane + 32 * k == p) {
             stuck |= 1u << k;
             if (full_receiver && native_big) slotlim |= 1u << k;
@@ -261,7 +286,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     unsigned wm = 0;
     bool sl = false;
 #pragma unroll
-    for (int k = 0; k < kRW; ++k)
+    for (int k = 0; k < RW; ++k)
       if (lane + 32 * k < R) {
         wm = max(wm, (unsigned)Wr[k]);
         sl |= ((stuck >> k) & 1u) && ((slotlim >> k) & 1u) && Wr[k] > C;
@@ -290,7 +315,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   __syncthreads();
   if (solver && j == s_best) {
 #pragma unroll
-    for (int k = 0; k < kRW; ++k) {
+    for (int k = 0; k < RW; ++k) {
       const int q = lane + 32 * k;
       if (q < R) {
         s_Wf[q] = Wr[k];
@@ -707,19 +732,19 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   int32_t* sg_base = sg_ord + segcap;                   // [segcap] row - ordinal
   int32_t* sg_rank = sg_base + segcap;                  // [segcap] destination rank
   int32_t* base0 = sg_rank + (PASS > 0 ? segcap : 0);   // [E]
-  const int per_warp = E + (PASS > 0 ? R + (kSubT * K + 3) / 4 : 0);
+  const int per_warp = E + (PASS > 0 ? R + (kPlanSubT * K + 3) / 4 : 0);
   int32_t* run = base0 + E + warp * per_warp;           // [E] running ordinals
   int32_t* wrun = run + E;                              // [R] running shared ordinals
-  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);   // [kSubT*K] destination ranks
+  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);   // [kPlanSubT*K] destination ranks
 
   // The first batch of ids is an input no kernel of the plan writes: fetch it
   // before waiting for the predecessor grid.
-  const int t0 = active ? sub * kSubT : 0, t1 = active ? min(d.T, t0 + kSubT) : 0;
+  const int t0 = active ? sub * kPlanSubT : 0, t1 = active ? min(d.T, t0 + kPlanSubT) : 0;
   const int a0 = t0 * K, a1 = t1 * K;
   const int64_t rbase = (int64_t)r * d.T * K;
-  int v[kBatch];
+  int v[kAsgBatch];
 #pragma unroll
-  for (int u = 0; u < kBatch; ++u) {
+  for (int u = 0; u < kAsgBatch; ++u) {
     const int idx = a0 + u * 32 + lane;
     v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
   }
@@ -788,13 +813,15 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   }
   const int32_t* cnt_r = s.sub_cnt + (int64_t)r * d.nsub * E;
   {
-    const int n = sub0 * E;
+    // blocks of this rank before this one: their per-block counts
+    const int32_t* blk_r = s.blk_cnt + (int64_t)r * nbpr * E;
+    const int n = (sub0 / kWarpsPerBlock) * E;
     for (int i = tid; i < n; i += nthr * 8) {
       int c[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int ii = i + u * nthr;
-        c[u] = ii < n ? cnt_r[ii] : 0;
+        c[u] = ii < n ? blk_r[ii] : 0;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -813,16 +840,16 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   __syncwarp();
 
   bool inconsistent = false;
-  for (int a = a0; a < a1; a += kBatch * 32) {
+  for (int a = a0; a < a1; a += kAsgBatch * 32) {
     if (a != a0) {
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
+      for (int u = 0; u < kAsgBatch; ++u) {
         const int idx = a + u * 32 + lane;
         v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
       }
     }
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
+    for (int u = 0; u < kAsgBatch; ++u) {
       if (a + u * 32 >= a1) break;
       const int idx = a + u * 32 + lane;
       const int e = (v[u] >= 0 && v[u] < E) ? v[u] : -1;
@@ -1027,7 +1054,7 @@ size_t solve_smem(const Dims& d) { return sizeof(int32_t) * ((size_t)d.E * (1 + 
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
   const size_t segcap = (size_t)seg_capacity(d);
-  const size_t per_warp = d.E + (pass > 0 ? d.R + (kSubT * d.K + 3) / 4 : 0);
+  const size_t per_warp = d.E + (pass > 0 ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
   return sizeof(int32_t) *
          ((d.E + 1) + segcap * (pass > 0 ? 3 : 2) + d.E + (size_t)kWarpsPerBlock * per_warp);
 }
@@ -1054,34 +1081,64 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
 
 // Allow every kernel the device's opt-in shared-memory maximum once, so that
 // plans of any shape can coexist (each launch still requests only its own size).
+template <int SMAX>
+cudaError_t allow_solve(int max_smem) {
+  cudaError_t e;
+  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 1>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 2>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 3>, max_smem)) != cudaSuccess) return e;
+  return allow_max_dynamic_smem(k_solve<SMAX, 4>, max_smem);
+}
+
 cudaError_t set_plan_attributes(int max_smem) {
   cudaError_t e;
-  if ((e = allow_max_dynamic_smem(k_solve<1>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_solve<2>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_solve<4>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_solve<8>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_solve<1>(max_smem)) != cudaSuccess) return e;
+  if ((e = allow_solve<2>(max_smem)) != cudaSuccess) return e;
+  if ((e = allow_solve<4>(max_smem)) != cudaSuccess) return e;
+  if ((e = allow_solve<8>(max_smem)) != cudaSuccess) return e;
   if ((e = allow_max_dynamic_smem(k_hist, max_smem)) != cudaSuccess) return e;
   if ((e = allow_max_dynamic_smem(k_assign<0>, max_smem)) != cudaSuccess) return e;
   if ((e = allow_max_dynamic_smem(k_assign<1>, max_smem)) != cudaSuccess) return e;
   return allow_max_dynamic_smem(k_assign<2>, max_smem);
 }
 
+template <int SMAX>
+cudaError_t launch_solve_rw(const Dims& d, const LayerBuf& L, const Scratch& s, cudaStream_t st) {
+  const size_t ss = solve_smem(d);
+  const unsigned nt = kMaxJ * 32;
+  const int rw = (d.R + 31) / 32;
+  if (rw <= 1) return launch_pdl(k_solve<SMAX, 1>, 1, nt, ss, st, d, L, s);
+  if (rw == 2) return launch_pdl(k_solve<SMAX, 2>, 1, nt, ss, st, d, L, s);
+  if (rw == 3) return launch_pdl(k_solve<SMAX, 3>, 1, nt, ss, st, d, L, s);
+  return launch_pdl(k_solve<SMAX, 4>, 1, nt, ss, st, d, L, s);
+}
+
+cudaError_t launch_solve(const Dims& d, const LayerBuf& L, const Scratch& s, cudaStream_t st) {
+  if (d.S <= 1) return launch_solve_rw<1>(d, L, s, st);
+  if (d.S <= 2) return launch_solve_rw<2>(d, L, s, st);
+  if (d.S <= 4) return launch_solve_rw<4>(d, L, s, st);
+  return launch_solve_rw<8>(d, L, s, st);
+}
+
 cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, const int32_t* ids,
                            cudaStream_t st) {
-  // stats, load matrix, expert totals and tickets are adjacent in the layer block
+  // stats, load matrix, expert totals and tickets are adjacent in the layer
+  // block (256-byte aligned pieces): one clearing kernel covers them
   const size_t zero_bytes = reinterpret_cast<const char*>(L.tickets + 4) -
                             reinterpret_cast<const char*>(L.stats);
-  cudaError_t err = cudaMemsetAsync(L.stats, 0, zero_bytes, st);
+  const int64_t n16 = (int64_t)((zero_bytes + 15) / 16);
+  const int64_t cblocks = (n16 + 255) / 256;
+  k_clear_layer<<<(unsigned)(cblocks < 64 ? cblocks : 64), 256, 0, st>>>(
+      reinterpret_cast<int4*>(L.stats), n16);
+  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const unsigned nblk = (unsigned)(d.R * ((d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock));
   const unsigned bt = kWarpsPerBlock * 32;
-  if (nblk > 0) k_hist<<<nblk, bt, hist_smem(d), st>>>(ids, d, s, L);
-  const size_t ss = solve_smem(d);
-  const unsigned sthreads = kMaxJ * 32;
-  if (d.S <= 1) err = launch_pdl(k_solve<1>, 1, sthreads, ss, st, d, L, s);
-  else if (d.S <= 2) err = launch_pdl(k_solve<2>, 1, sthreads, ss, st, d, L, s);
-  else if (d.S <= 4) err = launch_pdl(k_solve<4>, 1, sthreads, ss, st, d, L, s);
-  else err = launch_pdl(k_solve<8>, 1, sthreads, ss, st, d, L, s);
+  if (nblk > 0) {
+    err = launch_pdl(k_hist, nblk, bt, hist_smem(d), st, ids, d, s, L);
+    if (err != cudaSuccess) return err;
+  }
+  err = launch_solve(d, L, s, st);
   if (err != cudaSuccess) return err;
   err = launch_pdl(k_reroute, (unsigned)((d.E + kWarpsPerBlock - 1) / kWarpsPerBlock), bt, 0, st, d,
                    L, s);

@@ -127,6 +127,22 @@ class ClockSampler:
                 "samples": len(loaded)}
 
 
+def max_over_ranks(value, dist=None, device=None):
+    """The job's time for weak-scaled replicas: the largest per-rank device time."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank, ms):
+    """Whole-job units per second: every rank processes units_per_rank in ms."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def _dist_init():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -258,11 +274,7 @@ def run_gpu(args):
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
-    ms_total = t0.elapsed_time(t1)
-    if dist is not None:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     ms_step = ms_total / args.steps
     perm_ms = [a.elapsed_time(b) for a, b in perm_ev]
     perm_avg_ms = sum(perm_ms) / len(perm_ms)
@@ -307,12 +319,8 @@ def run_gpu(args):
             b.synchronize()
             if k >= 1:
                 e2e_ms.append(a.elapsed_time(b))
-        e2e_step = sum(e2e_ms) / len(e2e_ms)
-        if dist is not None:
-            tt = torch.tensor([e2e_step], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_step = float(tt.item())
-        e2e = {"value": world * w.A / (e2e_step * 1e-3), "unit": UNIT,
+        e2e_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms), dist, dev)
+        e2e = {"value": job_throughput(world, w.A, e2e_step), "unit": UNIT,
                "h2d_bytes_per_step": int(ids_np.nbytes + hidden.numel() * 2),
                "d2h_bytes_per_step": 64, "steps": args.e2e_steps, "ms_per_step": e2e_step}
         assert st["rows"] == stats["rows"]
@@ -334,7 +342,7 @@ def run_gpu(args):
     A = int(stats["assignments"])
     line = {
         "metric": METRIC,
-        "value": world * A / (ms_step * 1e-3),
+        "value": job_throughput(world, A, ms_step),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,

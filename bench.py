@@ -195,7 +195,8 @@ def _median(xs):
 
 
 def _balance_launches(w):
-    return 3 + (3 if w.shared_expert else 1)  # hist, solve, reroute + assign pass(es)
+    # clear, hist, solve, reroute + assign (or assign, shared scan, assign)
+    return 4 + (3 if w.shared_expert else 1)
 
 
 def _ratio(st, R):
@@ -261,7 +262,8 @@ def run_gpu(args):
     for _ in range(args.warmup):
         step()
     stats = plan.read_layer_stats(0)
-    launches_per_step = _balance_launches(w) + 4  # + stage, dispatch, re-stage, reduce
+    # + stage, dispatch, re-stage, reduce and its slot-clearing kernel
+    launches_per_step = _balance_launches(w) + 5
 
     # ---- timed region: K whole steps --------------------------------------
     perm_ev = [_events(torch) for _ in range(args.steps)]

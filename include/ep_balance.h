@@ -80,7 +80,8 @@ enum {
  *   1 <= R <= 128, 1 <= E <= 1024, natives per rank ceil(E/R) <= 32,
  *   1 <= K <= 16, T >= 0, R*T*(K+1) < 2^31, 0 <= S <= 8, m >= 1,
  *   1 <= J <= 16, hidden >= 8 with hidden*2 a multiple of 16 bytes,
- *   expert_weight_elems >= 0 and a multiple of 8, num_layers >= 1,
+ *   expert_weight_elems >= 0 and a multiple of 8,
+ *   R*S*ceil(expert_weight_elems/16) < 2^32, num_layers >= 1,
  *   0 <= waterfill_bonus_permille <= 1000.
  * Native placement is fixed: rank q hosts the contiguous block of experts
  * [q*(E/R) + min(q, E%R), ... + E/R + (q < E%R)) ([U] §"Shared redundant

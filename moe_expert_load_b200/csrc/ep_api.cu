@@ -58,6 +58,9 @@ ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
       c->expert_weight_elems % 8 != 0)
     return EP_ERR_UNSUPPORTED;
   if ((int64_t)R * T * (K + 1) >= (int64_t)INT32_MAX) return EP_ERR_UNSUPPORTED;
+  // the gradient reduction indexes (replica slot, 16-element pair) in 32 bits
+  if ((int64_t)R * c->slots_per_rank * ((c->expert_weight_elems + 15) / 16) >= ((int64_t)1 << 32))
+    return EP_ERR_UNSUPPORTED;
   // Waterfill draw weights stay below 2^32: (K + 2) * H with H <= ceil((A + N) / R) + 1
   const int64_t H = ((int64_t)T * (K + 1) * R + R - 1) / R + 1;
   if ((int64_t)(K + 2) * H >= ((int64_t)1 << 32)) return EP_ERR_UNSUPPORTED;

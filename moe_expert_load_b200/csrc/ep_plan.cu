@@ -125,6 +125,37 @@ __global__ void __launch_bounds__(256) k_clear_layer(int4* __restrict__ p, int64
     p[i] = make_int4(0, 0, 0, 0);
 }
 
+// Warp argmax over the ranks lane + 32k (k < RW) with ok[k] set: the largest
+// v, smallest rank on ties.  When every v is below 2^24 the value and the rank
+// travel in one key, v * 128 + (127 - rank), and one redux finds both;
+// otherwise a max redux and a ballot per word.  Returns vmax = 0 when no rank
+// is ok (the rank returned is then meaningless).
+template <int RW>
+__device__ __forceinline__ int warp_argmax_rank(const unsigned (&v)[RW], const bool (&ok)[RW],
+                                                bool pack, int lane, unsigned& vmax) {
+  if (pack) {
+    unsigned key = 0;
+#pragma unroll
+    for (int k = 0; k < RW; ++k)
+      if (ok[k]) key = max(key, (v[k] << 7) | (unsigned)(127 - (lane + 32 * k)));
+    key = __reduce_max_sync(kFull, key);
+    vmax = key >> 7;
+    return 127 - (int)(key & 127u);
+  }
+  unsigned mx = 0;
+#pragma unroll
+  for (int k = 0; k < RW; ++k)
+    if (ok[k]) mx = max(mx, v[k]);
+  vmax = __reduce_max_sync(kFull, mx);
+  int q = -1;
+#pragma unroll
+  for (int k = 0; k < RW; ++k) {
+    const unsigned b = __ballot_sync(kFull, ok[k] && v[k] == vmax);
+    if (q < 0 && b) q = 32 * k + __ffs(b) - 1;
+  }
+  return q;
+}
+
 // ---------------------------------------------------------------------------
 // a2: quota solve.  One CTA; warp j runs the greedy at cap
 // C_j = ceil(A (200 + j) / (200 R)).  Greedy step: the most-loaded rank p that is
@@ -198,33 +229,42 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     }
     __syncwarp();
     const int iter_cap = 4 * (R * S + R + E) + 64;
+    // every key value is a load, a slack or a quota: at most C <= 1.08 A
+    const bool pack = A < (1 << 24);
     for (int it = 0;; ++it) {
       if (it >= iter_cap) { stop = EP_STOP_ITER_CAP; break; }
-      unsigned lm = 0;
-#pragma unroll
-      for (int k = 0; k < RW; ++k)
-        if (lane + 32 * k < R && !((stuck >> k) & 1u)) lm = max(lm, (unsigned)Wr[k]);
-      const int vmax = (int)__reduce_max_sync(kFull, lm);
-      if (vmax <= C) break;
-      int p = -1;
+      unsigned wv[RW];
+      bool wok[RW];
 #pragma unroll
       for (int k = 0; k < RW; ++k) {
-        const unsigned b = __ballot_sync(
-            kFull, lane + 32 * k < R && !((stuck >> k) & 1u) && Wr[k] == vmax);
-        if (p < 0 && b) p = 32 * k + __ffs(b) - 1;
+        wv[k] = (unsigned)Wr[k];
+        wok[k] = lane + 32 * k < R && !((stuck >> k) & 1u);
       }
+      unsigned uvmax;
+      const int p = warp_argmax_rank<RW>(wv, wok, pack, lane, uvmax);
+      const int vmax = (int)uvmax;
+      if (vmax <= C) break;
       const int ex = vmax - C;
       const int nf = nat_first(p, E, R), nc = nat_count(p, E, R);
       const int myQ = lane < nc ? Qn[nf + lane] : 0;
       bool tried = false, moved = false;
       for (;;) {
+        // the donor's untried native with the largest quota >= m (smallest e on ties)
         const unsigned cq = (lane < nc && !tried && myQ >= m) ? (unsigned)myQ : 0u;
-        const unsigned qmax = __reduce_max_sync(kFull, cq);
+        unsigned qmax;
+        int li;
+        if (pack) {
+          const unsigned key = __reduce_max_sync(kFull, cq ? (cq << 5) | (unsigned)(31 - lane) : 0u);
+          qmax = key >> 5;
+          li = 31 - (int)(key & 31u);
+        } else {
+          qmax = __reduce_max_sync(kFull, cq);
+          li = __ffs(__ballot_sync(kFull, cq == qmax)) - 1;
+        }
         if (qmax == 0) break;
-        const int li = __ffs(__ballot_sync(kFull, cq == qmax)) - 1;
         const int e = nf + li;
         // receivers: free slot, no instance of e, slack >= m
-        unsigned ls = 0;
+        unsigned sv[RW];
         bool ok[RW];
 #pragma unroll
         for (int k = 0; k < RW; ++k) {
@@ -233,18 +273,22 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
 #pragma unroll
           for (int t = 0; t < SMAX; ++t) h |= (se[k][t] == e);
           ok[k] = q < R && q != p && used[k] < S && !h && C - Wr[k] >= m;
-          if (ok[k]) ls = max(ls, (unsigned)(C - Wr[k]));
+          sv[k] = (unsigned)(C - Wr[k]);
         }
-        const unsigned smax = __reduce_max_sync(kFull, ls);
+        unsigned smax;
+        const int rr = warp_argmax_rank<RW>(sv, ok, pack, lane, smax);
         if (smax == 0) {
           if (lane == li) tried = true;
-          continue;
-        }
-        int rr = -1;
+          // no rank other than p has a free slot and slack >= m at all: every
+          // other native fails the same way
+          bool any_r = false;
 #pragma unroll
-        for (int k = 0; k < RW; ++k) {
-          const unsigned b = __ballot_sync(kFull, ok[k] && (unsigned)(C - Wr[k]) == smax);
-          if (rr < 0 && b) rr = 32 * k + __ffs(b) - 1;
+          for (int k = 0; k < RW; ++k) {
+            const int q = lane + 32 * k;
+            any_r |= q < R && q != p && used[k] < S && C - Wr[k] >= m;
+          }
+          if (!__any_sync(kFull, any_r)) break;
+          continue;
         }
         const int x = min(min(max(ex, m), (int)smax), (int)qmax);
 #pragma unroll

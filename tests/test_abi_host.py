@@ -81,6 +81,17 @@ def test_config_validation(field, value, code):
     assert ei.value.status == code
 
 
+def test_reduction_index_limit():
+    # (replica slots) x (16-element pairs per expert) must stay below 2^32
+    c = config_from_workload(get_config("tiny"), num_ranks=128, slots_per_rank=8,
+                             expert_weight_elems=1 << 26)
+    with pytest.raises(EpError) as ei:
+        ep_plan_workspace_bytes(c)
+    assert ei.value.status == 2
+    c.expert_weight_elems = (1 << 26) - 16
+    assert ep_plan_workspace_bytes(c) > 0
+
+
 def test_natives_per_rank_limit():
     c = config_from_workload(get_config("tiny"), num_experts=33 * 4)
     with pytest.raises(EpError):

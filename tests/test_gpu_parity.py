@@ -26,6 +26,18 @@ def test_plan_parity_full_configs(name):
     compare_plan(fetch(plan), o, w)
 
 
+def test_plan_parity_large_counts():
+    # R*T*K = 2^24 assignments: load, slack and quota values too wide for the
+    # solver's one-redux argmax keys, so it takes the two-step (max, ballot) path
+    w = get_config("stress").replace(R=64, T=32768, S=2, distinct=True, hot_frac=None, seed=6001)
+    assert w.A == 1 << 24
+    ids = topk_ids(w)
+    o = oracle_plan(w, ids)
+    plan = gpu_plan(w, ids)
+    compare_plan(fetch(plan), o, w)
+    assert o.replicas > 0
+
+
 def test_plan_parity_sweep_layers_cached():
     w = get_config("sweep")
     layers = [0, 1, 3, 47, 93]
@@ -191,11 +203,13 @@ def test_stage_replicas_qwen():
 
 
 @pytest.mark.parametrize("grad_dtype", ["bf16", "f32"])
-def test_reduce_grads_bit_exact(grad_dtype):
-    w = get_config("dsv3").replace(ffn=9)  # small experts (ragged last chunk), same routing
-    ids = topk_ids(get_config("dsv3"))
-    plan = gpu_plan(w, ids)
-    Wn = w.expert_elems
+@pytest.mark.parametrize("Wn", [3 * 7168 * 9, 1000, 8])
+def test_reduce_grads_bit_exact(grad_dtype, Wn):
+    # small experts, same routing as dsv3; 1000 and 8 leave a lone 8-element
+    # vector at the end of each expert (Wn % 16 == 8)
+    w = get_config("dsv3")
+    ids = topk_ids(w)
+    plan = gpu_plan(w, ids, expert_weight_elems=Wn)
     rng = np.random.default_rng(3)
     g32 = (rng.standard_normal((w.R, w.S, Wn)) * 1e-2).astype(np.float32)
     if grad_dtype == "bf16":

@@ -194,6 +194,9 @@ def _median(xs):
     return xs[len(xs) // 2]
 
 
+E2E_CHUNKS = 8  # token chunks of the end-to-end step's hidden-state copy
+
+
 def _balance_launches(w):
     # clear, hist, solve, reroute + assign (or assign, shared scan, assign)
     return 4 + (3 if w.shared_expert else 1)
@@ -308,14 +311,33 @@ def run_gpu(args):
     if args.e2e_steps > 0:
         ids_h = torch.from_numpy(ids_np).pin_memory()
         hidden_h = hidden.cpu().pin_memory()
+        # the hidden states arrive in token chunks on a copy stream; each
+        # chunk is dispatched (ep_dispatch_tokens) as soon as it has landed
+        copy_stream = torch.cuda.Stream(device=dev)
+        bounds = [w.N * c // E2E_CHUNKS for c in range(E2E_CHUNKS + 1)]
         e2e_ms = []
         for k in range(args.e2e_steps + 1):
             barrier()
             a, b = _events(torch)
+            ids_ev = torch.cuda.Event()
+            chunk_ev = [torch.cuda.Event() for _ in range(E2E_CHUNKS)]
             a.record(stream)
-            ids.copy_(ids_h, non_blocking=True)
-            hidden.copy_(hidden_h, non_blocking=True)
-            step()
+            copy_stream.wait_stream(stream)  # the previous step is done with the buffers
+            with torch.cuda.stream(copy_stream):
+                ids.copy_(ids_h, non_blocking=True)
+                ids_ev.record(copy_stream)
+                for c in range(E2E_CHUNKS):
+                    lo, hi = bounds[c], bounds[c + 1]
+                    hidden[lo:hi].copy_(hidden_h[lo:hi], non_blocking=True)
+                    chunk_ev[c].record(copy_stream)
+            stream.wait_event(ids_ev)
+            plan.balance_layer(0, ids)
+            plan.stage_replicas(0, native_w, slots)
+            for c in range(E2E_CHUNKS):
+                stream.wait_event(chunk_ev[c])
+                plan.dispatch_tokens(0, hidden, out, bounds[c], bounds[c + 1])
+            plan.stage_replicas(0, native_w, slots)
+            plan.reduce_replica_grads(0, slot_grads, native_grads)
             st = plan.read_layer_stats(0)  # device -> host read of the step's result
             b.record(stream)
             b.synchronize()
@@ -324,7 +346,8 @@ def run_gpu(args):
         e2e_step = max_over_ranks(sum(e2e_ms) / len(e2e_ms), dist, dev)
         e2e = {"value": job_throughput(world, w.A, e2e_step), "unit": UNIT,
                "h2d_bytes_per_step": int(ids_np.nbytes + hidden.numel() * 2),
-               "d2h_bytes_per_step": 64, "steps": args.e2e_steps, "ms_per_step": e2e_step}
+               "d2h_bytes_per_step": 64, "steps": args.e2e_steps, "ms_per_step": e2e_step,
+               "h2d_chunks": E2E_CHUNKS}
         assert st["rows"] == stats["rows"]
 
     if dist is not None:

@@ -196,6 +196,24 @@ EP_API ep_status_t ep_dispatch_layout(ep_plan* plan, int32_t layer, const void* 
                                int32_t dst_rank_end, void* stream);
 
 /*
+ * Token-range dispatch: the rows of source tokens n in [token_begin,
+ * token_end) only (n = r*T + t), for every destination rank:
+ * out[row] = hidden[n] for each dispatch row (routed and shared) of those
+ * tokens; rows of other tokens are not touched.  The pages have no
+ * counterpart: it lets a caller dispatch the tokens whose hidden states have
+ * arrived while the rest are still being copied in.  d_hidden is the whole
+ * [R*T][hidden] buffer (only the range's rows are read); d_out holds the whole
+ * layout (rows_total rows), out_rows_capacity its size in rows (rows beyond it
+ * are skipped and flag EP_DEV_OUT_CAPACITY).  An empty range does nothing.
+ * Errors: EP_ERR_INVALID_ARGUMENT for token_begin < 0, token_end > R*T,
+ * token_begin > token_end, a null or non-16-byte-aligned buffer (for a
+ * non-empty range); EP_ERR_NOT_PLANNED before ep_balance_layer.
+ */
+EP_API ep_status_t ep_dispatch_tokens(ep_plan* plan, int32_t layer, const void* d_hidden,
+                               int64_t token_begin, int64_t token_end, void* d_out,
+                               int64_t out_rows_capacity, void* stream);
+
+/*
  * Replica weight staging ([U] §"Shared redundant slots": hot experts' weights
  * are written into the reserved slots, shared by all layers; backward re-stages
  * from the cached forward plan): d_slots[q][s] = d_native_w[expert of slot (q,s)]

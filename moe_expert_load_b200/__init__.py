@@ -8,6 +8,7 @@ the library is not built, importing the entry points raises (no fallback).
     plan = Plan(config_from_workload(get_config("qwen")))
     plan.balance_layer(0, ids)                  # ep_balance_layer
     out = plan.dispatch_layout(0, hidden)       # ep_dispatch_layout
+    plan.dispatch_tokens(0, hidden, out, 0, n)  # ep_dispatch_tokens (source-token range)
     plan.stage_replicas(0, native_w, slots)     # ep_stage_replicas
     plan.reduce_replica_grads(0, g_slots, g_native)
 """
@@ -168,6 +169,14 @@ class Plan:
             out = torch.empty((out_rows, hidden.shape[1]), dtype=hidden.dtype, device=hidden.device)
         _check("ep_dispatch_layout", self.lib.ep_dispatch_layout(
             self.handle, layer, _ptr(hidden), _ptr(out), out.shape[0], rank_begin, rank_end, _stream(stream)))
+        return out
+
+    def dispatch_tokens(self, layer: int, hidden: torch.Tensor, out: torch.Tensor, token_begin: int,
+                        token_end: int, stream=None) -> torch.Tensor:
+        """ep_dispatch_tokens: every dispatch row of source tokens [token_begin, token_end)."""
+        _check("ep_dispatch_tokens", self.lib.ep_dispatch_tokens(
+            self.handle, layer, _ptr(hidden), token_begin, token_end, _ptr(out), out.shape[0],
+            _stream(stream)))
         return out
 
     def combine(self, layer: int, expert_out: torch.Tensor, weights: torch.Tensor,

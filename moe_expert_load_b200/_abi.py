@@ -27,7 +27,7 @@ EXPORTS = (
     "ep_plan_workspace_bytes", "ep_plan_create", "ep_plan_destroy", "ep_balance_layer",
     "ep_layer_view_get", "ep_read_layer_stats", "ep_dispatch_layout", "ep_stage_replicas",
     "ep_reduce_replica_grads", "ep_waterfill", "ep_status_string", "ep_abi_version",
-    "ep_load_matrix_static", "ep_combine",
+    "ep_load_matrix_static", "ep_combine", "ep_dispatch_tokens",
 )
 
 
@@ -100,6 +100,7 @@ def load():
         "ep_layer_view_get": (S, [P, I32, ctypes.POINTER(EpLayerView)]),
         "ep_read_layer_stats": (S, [P, I32, ctypes.POINTER(EpLayerStats), P]),
         "ep_dispatch_layout": (S, [P, I32, P, P, I64, I32, I32, P]),
+        "ep_dispatch_tokens": (S, [P, I32, P, I64, I64, P, I64, P]),
         "ep_stage_replicas": (S, [P, I32, P, P, P]),
         "ep_reduce_replica_grads": (S, [P, I32, P, I32, P, P]),
         "ep_waterfill": (S, [I32, I32, I32, P, P, ctypes.c_uint64, I32, I32, P, P, P]),

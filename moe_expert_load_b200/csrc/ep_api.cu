@@ -334,7 +334,24 @@ ep_status_t ep_dispatch_layout(ep_plan* plan, int32_t layer, const void* d_hidde
   if (!aligned16(d_hidden) || !aligned16(d_out)) return EP_ERR_INVALID_ARGUMENT;
   if (dst_rank_begin == dst_rank_end) return EP_OK;
   return cuda_status(ep::launch_dispatch(plan->d, layer_buf(plan, layer), d_hidden, d_out,
-                                         out_rows_capacity, dst_rank_begin, dst_rank_end,
+                                         out_rows_capacity, dst_rank_begin, dst_rank_end, 0,
+                                         (int64_t)plan->d.R * plan->d.T, plan->num_sms,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_dispatch_tokens(ep_plan* plan, int32_t layer, const void* d_hidden, int64_t token_begin,
+                               int64_t token_end, void* d_out, int64_t out_rows_capacity,
+                               void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!plan->planned[layer]) return EP_ERR_NOT_PLANNED;
+  const int64_t N = (int64_t)plan->d.R * plan->d.T;
+  if (token_begin < 0 || token_end > N || token_begin > token_end || out_rows_capacity < 0)
+    return EP_ERR_INVALID_ARGUMENT;
+  if (token_begin == token_end) return EP_OK;
+  if (!d_hidden || !d_out || !aligned16(d_hidden) || !aligned16(d_out)) return EP_ERR_INVALID_ARGUMENT;
+  return cuda_status(ep::launch_dispatch(plan->d, layer_buf(plan, layer), d_hidden, d_out,
+                                         out_rows_capacity, 0, plan->d.R, token_begin, token_end,
                                          plan->num_sms, static_cast<cudaStream_t>(stream)));
 }
 

@@ -44,7 +44,7 @@ struct PermuteArgs {
   const int32_t* shared_row;  // null without a shared expert
   const int32_t* rank_base;
   ep_layer_stats* stats;
-  int64_t N;
+  int64_t n0, N;  // tokens [n0, N)
   int64_t cap_rows;
   int row16;  // 16-byte words per row
   int K;
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kPermuteThreads) k_permute(PermuteArgs a) {
   const int row_hi = a.rank_base[a.rank_end];
   const int row16 = a.row16;
   bool overflow = false;
-  for (int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < a.N; n += nw) {
+  for (int64_t n = a.n0 + (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); n < a.N; n += nw) {
     int d = -1;
     if (lane < a.K) d = a.dst_row[n * a.K + lane];
     else if (lane == a.K && a.shared_row != nullptr) d = a.shared_row[n];
@@ -413,8 +413,8 @@ cudaError_t set_copy_attributes(int max_smem) {
 }
 
 cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden, void* out,
-                            int64_t cap_rows, int rank_begin, int rank_end, int num_sms,
-                            cudaStream_t st) {
+                            int64_t cap_rows, int rank_begin, int rank_end, int64_t token_begin,
+                            int64_t token_end, int num_sms, cudaStream_t st) {
   PermuteArgs a;
   a.hidden = static_cast<const uint4*>(hidden);
   a.out = static_cast<uint4*>(out);
@@ -422,16 +422,21 @@ cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden
   a.shared_row = d.sh ? L.shared_row : nullptr;
   a.rank_base = L.rank_base;
   a.stats = L.stats;
-  a.N = (int64_t)d.R * d.T;
+  a.n0 = token_begin;
+  a.N = token_end;
   a.cap_rows = cap_rows;
   a.row16 = d.hidden * 2 / 16;
   a.K = d.K;
   a.rank_begin = rank_begin;
   a.rank_end = rank_end;
-  if (a.N == 0) return cudaSuccess;
+  if (a.N <= a.n0) return cudaSuccess;
   // 12 blocks of 4 warps per SM, about twice what is resident at once:
-  // measured 6.0 (8), 6.1-6.2 (12) and 6.1 (16) TB/s on the qwen layer
-  k_permute<<<(unsigned)(num_sms * 12), kPermuteThreads, 0, st>>>(a);
+  // measured 6.0 (8), 6.1-6.2 (12) and 6.1 (16) TB/s on the qwen layer;
+  // a short token range needs no more than one warp per token
+  const int64_t warps = (a.N - a.n0);
+  const int64_t blocks = (warps + kPermuteThreads / 32 - 1) / (kPermuteThreads / 32);
+  const int64_t grid = blocks < (int64_t)num_sms * 12 ? blocks : (int64_t)num_sms * 12;
+  k_permute<<<(unsigned)grid, kPermuteThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

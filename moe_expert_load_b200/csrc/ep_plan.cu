@@ -174,6 +174,8 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   int32_t* Tot = sm;              // [E]
   int32_t* Qn_all = sm + d.E;     // [J][E]
   int32_t* cnt_e = Qn_all + d.J * d.E;  // [E+1]
+  int32_t* s_eptr = cnt_e + d.E + 1;    // [E+1] replica-list offsets
+  int32_t* s_rel = s_eptr + d.E + 1;    // [R*G] rank-relative first rows
   __shared__ int32_t s_W0[kMaxR];
   __shared__ int32_t s_Wf[kMaxR];
   __shared__ int32_t s_se[kMaxR * kMaxS];
@@ -350,11 +352,13 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     }
   }
   __syncthreads();
-  if (tid == 0) {  // smallest (max load, replicas, j)
-    int b = 0;
-    for (int jj = 1; jj < d.J; ++jj)
-      if (s_cmax[jj] < s_cmax[b] || (s_cmax[jj] == s_cmax[b] && s_crep[jj] < s_crep[b])) b = jj;
-    s_best = b;
+  if (warp == 0) {  // smallest (max load, replicas, j)
+    const unsigned k1 = lane < d.J ? (unsigned)s_cmax[lane] : 0xffffffffu;
+    const unsigned m1 = __reduce_min_sync(kFull, k1);
+    const unsigned k2 = (lane < d.J && k1 == m1) ? (unsigned)s_crep[lane] * 32u + (unsigned)lane
+                                                 : 0xffffffffu;
+    const unsigned m2 = __reduce_min_sync(kFull, k2);
+    if (lane == 0) s_best = (int)(m2 & 31u);
   }
   __syncthreads();
   if (solver && j == s_best) {
@@ -406,6 +410,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     int run = 0;
     for (int col = 0; col < G; ++col) {
       s.inst_rel[tid * G + col] = run;
+      s_rel[tid * G + col] = run;
       int qu = 0;
       if (col < Gmax) {
         if (col < nat_count(tid, E, R)) qu = Qw[nat_first(tid, E, R) + col];
@@ -436,7 +441,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   }
   __syncthreads();
   if (!d.sh) {
-    for (int i = tid; i < R * G; i += nthr) L.inst_off[i] = s_base[i / G] + s.inst_rel[i];
+    for (int i = tid; i < R * G; i += nthr) L.inst_off[i] = s_base[i / G] + s_rel[i];
     if (tid == 0) L.inst_off[R * G] = s_base[R];
     for (int q = tid; q <= R; q += nthr) L.rank_base[q] = s_base[q];
     if (tid == 0) L.stats->rows = s_base[R];
@@ -470,7 +475,10 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
         const int z = __shfl_up_sync(kFull, fincl, o);
         if (lane >= o) { incl += y; fincl += z; }
       }
-      if (e <= E) L.rep_eptr[e] = carry + incl - v;
+      if (e <= E) {
+        L.rep_eptr[e] = carry + incl - v;
+        s_eptr[e] = carry + incl - v;
+      }
       if (e < E && f) L.rep_experts[ncarry + fincl - 1] = e;
       carry += __shfl_sync(kFull, incl, 31);
       ncarry += __shfl_sync(kFull, fincl, 31);
@@ -483,7 +491,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     if (e < 0) continue;
     int before = 0;
     for (int i2 = 0; i2 < i; ++i2) before += (s_se[i2] == e);
-    L.rep_list[L.rep_eptr[e] + before] = i;
+    L.rep_list[s_eptr[e] + before] = i;
   }
 }
 
@@ -1094,7 +1102,9 @@ k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
   atomicAdd(&count[c], 1);
 }
 
-size_t solve_smem(const Dims& d) { return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + d.E + 1); }
+size_t solve_smem(const Dims& d) {
+  return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + 2 * ((size_t)d.E + 1) + (size_t)d.R * d.G);
+}
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
   const size_t segcap = (size_t)seg_capacity(d);

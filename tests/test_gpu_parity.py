@@ -161,6 +161,55 @@ def test_dispatch_rank_windows_concatenate():
     assert plan.read_layer_stats(0)["status"] == 0
 
 
+@pytest.mark.parametrize("shared", [False, True])
+def test_dispatch_token_ranges_match_oracle(shared):
+    # ragged source-token chunks, each written into the same buffer, give the
+    # oracle's permutation; a chunk writes only its own tokens' rows
+    w = get_config("tiny").replace(T=777, shared_expert=shared)
+    ids = topk_ids(get_config("tiny"))[:, :777].copy()
+    plan = gpu_plan(w, ids)
+    hidden = _hidden(w, 2)
+    o = oracle_plan(w, ids)
+    want = oracle.permute(o, hidden.view(torch.int16).cpu().numpy())
+    rows = w.A + (w.N if shared else 0)
+    out = torch.zeros((rows, w.hidden), dtype=torch.bfloat16, device="cuda")
+    cuts = [0, 1, 500, 2047, 2048, 3000, w.N]
+    plan.dispatch_tokens(0, hidden, out, 500, 2047)
+    torch.cuda.synchronize()
+    got = out.view(torch.int16).cpu().numpy()
+    mine = np.zeros(rows, bool)
+    dst = o.dst_row.reshape(w.N, w.K)[500:2047]
+    mine[dst.ravel()] = True
+    if shared:
+        mine[o.shared_row.reshape(w.N)[500:2047]] = True
+    np.testing.assert_array_equal(got[mine], want[mine])
+    assert not got[~mine].any()
+    for b, e in zip(cuts[:-1], cuts[1:]):
+        plan.dispatch_tokens(0, hidden, out, b, e)
+    plan.dispatch_tokens(0, hidden, out, 7, 7)  # empty range: nothing
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.view(torch.int16).cpu().numpy(), want)
+    assert plan.read_layer_stats(0)["status"] == 0
+
+
+def test_dispatch_tokens_argument_errors():
+    w = get_config("tiny")
+    plan = Plan(config_from_workload(w))
+    hidden = _hidden(w)
+    out = torch.empty((w.A, w.hidden), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(EpError) as ei:
+        plan.dispatch_tokens(0, hidden, out, 0, 10)
+    assert ei.value.status == 5  # not planned yet
+    plan.balance_layer(0, torch.from_numpy(topk_ids(w)).cuda())
+    for b, e in [(-1, 3), (5, 4), (0, w.N + 1)]:
+        with pytest.raises(EpError) as ei:
+            plan.dispatch_tokens(0, hidden, out, b, e)
+        assert ei.value.status == 1
+    plan.dispatch_tokens(0, hidden, out, 0, w.N)
+    torch.cuda.synchronize()
+    assert plan.read_layer_stats(0)["status"] == 0
+
+
 def test_dispatch_capacity_overflow_is_flagged_not_written():
     w = get_config("tiny")
     ids = topk_ids(w)

@@ -187,6 +187,9 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int R = d.R, E = d.E, S = d.S, m = d.m;
+  // native placement: rank q holds [q*eb + min(q, er), +eb + (q < er)); one
+  // division here rather than one per greedy step
+  const int eb = E / R, er = E - (E / R) * R;
 
   pdl_trigger();
   pdl_wait();
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   if (tid == 0) s_iter_cap_hit = 0;
   __syncthreads();
   if (tid < R) {
-    const int f = nat_first(tid, E, R), n = nat_count(tid, E, R);
+    const int f = tid * eb + min(tid, er), n = eb + (tid < er ? 1 : 0);
     int w = 0;
     for (int i = 0; i < n; ++i) w += Tot[f + i];
     s_W0[tid] = w;
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       const int vmax = (int)uvmax;
       if (vmax <= C) break;
       const int ex = vmax - C;
-      const int nf = nat_first(p, E, R), nc = nat_count(p, E, R);
+      const int nf = p * eb + min(p, er), nc = eb + (p < er ? 1 : 0);
       const int myQ = lane < nc ? Qn[nf + lane] : 0;
       bool tried = false, moved = false;
       for (;;) {
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     const int q = i / G, col = i - (i / G) * G;
     int ex = -1, qu = 0;
     if (col < Gmax) {
-      if (col < nat_count(q, E, R)) { ex = nat_first(q, E, R) + col; qu = Qw[ex]; }
+      if (col < eb + (q < er ? 1 : 0)) { ex = q * eb + min(q, er) + col; qu = Qw[ex]; }
     } else if (col < Gmax + S) {
       ex = s_se[q * S + col - Gmax];
       qu = s_sq[q * S + col - Gmax];
@@ -413,7 +416,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       s_rel[tid * G + col] = run;
       int qu = 0;
       if (col < Gmax) {
-        if (col < nat_count(tid, E, R)) qu = Qw[nat_first(tid, E, R) + col];
+        if (col < eb + (tid < er ? 1 : 0)) qu = Qw[tid * eb + min(tid, er) + col];
       } else if (col < Gmax + S) {
         qu = s_sq[tid * S + col - Gmax];
       }

@@ -11,6 +11,7 @@
 // Everything is integer arithmetic; all orders are fixed, so results are
 // bit-identical run to run and independent of the grid size.
 #include <cuda_runtime.h>
+#include <limits.h>
 #include <stdint.h>
 
 #include "ep_internal.cuh"
@@ -750,12 +751,14 @@ __device__ __forceinline__ int wf_pick(int r, int64_t token, const unsigned (&ma
 // ---------------------------------------------------------------------------
 // a4 (+a5): token assignment.  A block owns up to 8 consecutive sub-chunks of
 // one source rank r (one per warp).  It first copies rank r's rerouting
-// segments into shared memory — for each expert, (first ordinal, row offset,
-// destination rank) — and the exclusive base of its first sub-chunk, the sum
-// of the rank's earlier sub-chunk counts.  The stable ordinal of (t, k) among
-// rank r's assignments of expert e = that base + the counts of the block's
-// earlier warps + the warp's running count + the rank inside the 32-lane
-// match.any group; the ordinal selects the segment and thus the row.
+// segments into shared memory — for each segment (first ordinal, row offset,
+// destination rank), and per expert one 16-byte record holding its first
+// segment and where the second begins, so that most lookups are one load —
+// and the exclusive base of its first sub-chunk, the sum of the rank's earlier
+// blocks' totals.  The stable ordinal of (t, k) among rank r's assignments of
+// expert e = that base + the counts of the block's earlier warps + the warp's
+// running count + the rank inside the 32-lane match.any group; the ordinal
+// selects the segment and thus the row.
 // PASS 0: rows, no shared expert.  PASS 1: Waterfill picks, counted per
 // (destination rank, sub-chunk).  PASS 2: rows and shared-slot rows.
 // ---------------------------------------------------------------------------
@@ -768,7 +771,7 @@ __host__ __device__ __forceinline__ int seg_capacity(const Dims& d) {
 template <int PASS>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
-  extern __shared__ int32_t sm[];
+  extern __shared__ __align__(16) int32_t sm[];
   __shared__ int32_t s_slack[kMaxR];
   __shared__ int32_t s_W[kMaxR];
   __shared__ int32_t s_sbase[kMaxR];
@@ -782,8 +785,10 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   const int sub = sub0 + warp;
   const bool active = sub < d.nsub;
   const int segcap = seg_capacity(d);
-  int32_t* sg_lo = sm;                                  // [E+1]
-  int32_t* sg_ord = sg_lo + E + 1;                      // [segcap] first ordinal
+  // per expert: {first segment, segment count | first segment's rank << 16,
+  // first segment's row - ordinal, second segment's first ordinal (or INT_MAX)}
+  int4* sge = reinterpret_cast<int4*>(sm);              // [E]
+  int32_t* sg_ord = sm + 4 * E;                         // [segcap] first ordinal
   int32_t* sg_base = sg_ord + segcap;                   // [segcap] row - ordinal
   int32_t* sg_rank = sg_base + segcap;                  // [segcap] destination rank
   int32_t* base0 = sg_rank + (PASS > 0 ? segcap : 0);   // [E]
@@ -838,14 +843,22 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     for (int u = 0; u < 4; ++u) {
       const int e = eb + u;
       if (u < per && e < E) {
-        sg_lo[e] = off;
         const int64_t gb = (int64_t)e * 3 * R + s0[u];
+        int4 g = make_int4(off, 0, 0, INT_MAX);
         for (int j = 0; j < cnt[u] && off + j < segcap; ++j) {
           const int ord = s.seg_ord[gb + j], rank = s.seg_rank[gb + j];
+          const int base = PASS != 1 ? L.rank_base[rank] + s.seg_rel[gb + j] - ord : 0;
           sg_ord[off + j] = ord;
-          if (PASS != 1) sg_base[off + j] = L.rank_base[rank] + s.seg_rel[gb + j] - ord;
+          if (PASS != 1) sg_base[off + j] = base;
           if (PASS > 0) sg_rank[off + j] = rank;
+          if (j == 0) {
+            g.y = cnt[u] | (rank << 16);
+            g.z = base;
+          } else if (j == 1) {
+            g.w = ord;
+          }
         }
+        sge[e] = g;
         off += cnt[u];
       }
     }
@@ -860,7 +873,6 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     }
   }
   __syncthreads();
-  if (tid == 0) sg_lo[E] = s_total;
   const bool overflow = s_total > segcap;
   if (overflow) {
     if (tid == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
@@ -917,12 +929,18 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
       if (idx < a1) {
         int row = -1, rank = kNoRank;
         if (e >= 0) {
-          const int lo = sg_lo[e], hi = sg_lo[e + 1];
-          int si = hi - 1;
-          while (si > lo && sg_ord[si] > o) --si;
-          if (hi > lo) {
-            if (PASS != 1) row = sg_base[si] + o;
-            if (PASS > 0) rank = sg_rank[si];
+          const int4 g = sge[e];
+          const int n = g.y & 0xffff;
+          if (n > 0) {
+            int b = g.z, q = g.y >> 16;
+            if (o >= g.w) {  // a later segment: the last one starting at or before o
+              int si = g.x + n - 1;
+              while (si > g.x && sg_ord[si] > o) --si;
+              if (PASS != 1) b = sg_base[si];
+              if (PASS > 0) q = sg_rank[si];
+            }
+            if (PASS != 1) row = b + o;
+            if (PASS > 0) rank = q;
           } else {
             inconsistent = true;
           }
@@ -1113,7 +1131,7 @@ size_t assign_smem(const Dims& d, int pass) {
   const size_t segcap = (size_t)seg_capacity(d);
   const size_t per_warp = d.E + (pass > 0 ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
   return sizeof(int32_t) *
-         ((d.E + 1) + segcap * (pass > 0 ? 3 : 2) + d.E + (size_t)kWarpsPerBlock * per_warp);
+         (4 * (size_t)d.E + segcap * (pass > 0 ? 3 : 2) + d.E + (size_t)kWarpsPerBlock * per_warp);
 }
 
 // Launch with programmatic stream serialisation: the kernel may begin while

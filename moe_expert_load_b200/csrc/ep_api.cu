@@ -28,7 +28,7 @@ struct Layout {
   size_t layer_bytes;
   // scratch (absolute)
   size_t sub_cnt, blk_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase,
-      shared_tot;
+      shared_tot, asg_rank;
   size_t scratch_bytes;
   size_t total;
 };
@@ -121,6 +121,7 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.wf = s.take(i4 * 2);
   L.sbase = s.take(i4 * d.R);
   L.shared_tot = s.take(i4 * d.R);
+  L.asg_rank = s.take(d.sh ? (size_t)d.R * d.T * d.K : 0);
   L.total = s.off;
   L.scratch_bytes = s.off - L.layer_bytes * (size_t)num_layers;
   return L;
@@ -185,6 +186,7 @@ ep::Scratch scratch(const ep_plan* p) {
   s.wf = at(p, l.wf);
   s.sbase = at(p, l.sbase);
   s.shared_tot = at(p, l.shared_tot);
+  s.asg_rank = p->d.sh ? reinterpret_cast<uint8_t*>(p->ws + l.asg_rank) : nullptr;
   return s;
 }
 

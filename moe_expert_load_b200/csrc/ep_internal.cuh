@@ -70,6 +70,7 @@ struct Scratch {
   int32_t* wf;        // [2] Waterfill H, B
   int32_t* sbase;     // [R] first row of each rank's shared column
   int32_t* shared_tot;  // [R] shared-slot rows per destination rank
+  uint8_t* asg_rank;    // [R][T][K] destination rank of each assignment (shared expert only)
 };
 
 // ---- native placement: contiguous balanced blocks ---------------------------

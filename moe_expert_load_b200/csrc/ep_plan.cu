@@ -759,8 +759,11 @@ __device__ __forceinline__ int wf_pick(int r, int64_t token, const unsigned (&ma
 // expert e = that base + the counts of the block's earlier warps + the warp's
 // running count + the rank inside the 32-lane match.any group; the ordinal
 // selects the segment and thus the row.
-// PASS 0: rows, no shared expert.  PASS 1: Waterfill picks, counted per
-// (destination rank, sub-chunk).  PASS 2: rows and shared-slot rows.
+// PASS 0 (no shared expert): rows.  PASS 1 (shared expert): rows relative to
+// the destination rank's block and the destination ranks, then the Waterfill
+// pick of every token, its ordinal among the sub-chunk's tokens with that pick,
+// and the sub-chunk's pick counts per destination rank; k_fixup adds the rank
+// bases once the shared columns are laid out.
 // ---------------------------------------------------------------------------
 __host__ __device__ __forceinline__ int seg_capacity(const Dims& d) {
   // per source rank: at most one local segment per expert, and the remote
@@ -774,7 +777,6 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   extern __shared__ __align__(16) int32_t sm[];
   __shared__ int32_t s_slack[kMaxR];
   __shared__ int32_t s_W[kMaxR];
-  __shared__ int32_t s_sbase[kMaxR];
   __shared__ int32_t s_wsum[kWarpsPerBlock];
   __shared__ int32_t s_total;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
@@ -847,9 +849,9 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
         int4 g = make_int4(off, 0, 0, INT_MAX);
         for (int j = 0; j < cnt[u] && off + j < segcap; ++j) {
           const int ord = s.seg_ord[gb + j], rank = s.seg_rank[gb + j];
-          const int base = PASS != 1 ? L.rank_base[rank] + s.seg_rel[gb + j] - ord : 0;
+          const int base = (PASS == 0 ? L.rank_base[rank] : 0) + s.seg_rel[gb + j] - ord;
           sg_ord[off + j] = ord;
-          if (PASS != 1) sg_base[off + j] = base;
+          sg_base[off + j] = base;
           if (PASS > 0) sg_rank[off + j] = rank;
           if (j == 0) {
             g.y = cnt[u] | (rank << 16);
@@ -869,7 +871,7 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     if (PASS > 0) {
       s_slack[q] = s.slack[q];
       s_W[q] = L.W[q];
-      if (PASS == 2) s_sbase[q] = s.sbase[q];
+
     }
   }
   __syncthreads();
@@ -936,25 +938,27 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
             if (o >= g.w) {  // a later segment: the last one starting at or before o
               int si = g.x + n - 1;
               while (si > g.x && sg_ord[si] > o) --si;
-              if (PASS != 1) b = sg_base[si];
+              b = sg_base[si];
               if (PASS > 0) q = sg_rank[si];
             }
-            if (PASS != 1) row = b + o;
+            row = b + o;
             if (PASS > 0) rank = q;
           } else {
             inconsistent = true;
           }
         }
-        if (PASS != 1) L.dst_row[rbase + idx] = row;
-        if (PASS > 0) dr[idx - a0] = (uint8_t)rank;
+        L.dst_row[rbase + idx] = row;
+        if (PASS > 0) {
+          dr[idx - a0] = (uint8_t)rank;
+          s.asg_rank[rbase + idx] = (uint8_t)rank;
+        }
       }
     }
   }
   if (__any_sync(kFull, inconsistent) && lane == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
   if (PASS > 0) {
     const int gw = r * d.nsub + sub;
-    for (int q = lane; q < R; q += 32)
-      wrun[q] = PASS == 1 ? 0 : s.wsub_cnt[(int64_t)q * R * d.nsub + gw];
+    for (int q = lane; q < R; q += 32) wrun[q] = 0;
     __syncwarp();
     const int B = s.wf[1];
     for (int t = t0; t < t1; t += 32) {
@@ -979,15 +983,13 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
       __syncwarp();
       if (c >= 0 && lane == __ffs(peers) - 1) wrun[c] = o + __popc(peers);
       __syncwarp();
-      if (PASS == 2 && tt < t1) {
+      if (tt < t1) {
         L.shared_rank[(int64_t)r * d.T + tt] = c;
-        L.shared_row[(int64_t)r * d.T + tt] = s_sbase[c] + o;
+        L.shared_row[(int64_t)r * d.T + tt] = o;  // ordinal inside (c, sub-chunk) for now
       }
     }
-    if (PASS == 1) {
-      __syncwarp();
-      for (int q = lane; q < R; q += 32) s.wsub_cnt[(int64_t)q * R * d.nsub + gw] = wrun[q];
-    }
+    __syncwarp();
+    for (int q = lane; q < R; q += 32) s.wsub_cnt[(int64_t)q * R * d.nsub + gw] = wrun[q];
   }
 }
 
@@ -1084,6 +1086,54 @@ __global__ void __launch_bounds__(kScanThreads) k_shared_scan(Dims d, LayerBuf L
   }
 }
 
+// Shared expert, once the shared columns are laid out: every routed row gets
+// its destination rank's first row added, and every shared-slot row (still
+// the token's ordinal among its sub-chunk's tokens with the same pick) gets
+// its column's first row plus the picks of that rank in earlier (source rank,
+// sub-chunk) pairs.  Elementwise; four routed rows per 16-byte access.
+constexpr int kFixThreads = 256;
+
+__global__ void __launch_bounds__(kFixThreads) k_fixup(Dims d, LayerBuf L, Scratch s) {
+  __shared__ int32_t s_rb[kMaxR + 1];
+  __shared__ int32_t s_sb[kMaxR];
+  pdl_trigger();
+  pdl_wait();
+  const int R = d.R;
+  for (int q = threadIdx.x; q <= R; q += blockDim.x) {
+    s_rb[q] = L.rank_base[q];
+    if (q < R) s_sb[q] = s.sbase[q];
+  }
+  __syncthreads();
+  const int64_t A = (int64_t)R * d.T * d.K;
+  const int N = R * d.T;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  // dst_row and the rank bytes both start 256-byte aligned
+  const int64_t A4 = A / 4;
+  int4* row4 = reinterpret_cast<int4*>(L.dst_row);
+  const uint32_t* rk4 = reinterpret_cast<const uint32_t*>(s.asg_rank);
+  for (int64_t i = i0; i < A4; i += stride) {
+    int4 v = row4[i];
+    const uint32_t q = rk4[i];
+    const int q0 = q & 0xffu, q1 = (q >> 8) & 0xffu, q2 = (q >> 16) & 0xffu, q3 = q >> 24;
+    if (q0 != kNoRank) v.x += s_rb[q0];
+    if (q1 != kNoRank) v.y += s_rb[q1];
+    if (q2 != kNoRank) v.z += s_rb[q2];
+    if (q3 != kNoRank) v.w += s_rb[q3];
+    row4[i] = v;
+  }
+  for (int64_t i = 4 * A4 + i0; i < A; i += stride) {
+    const int q = s.asg_rank[i];
+    if (q != kNoRank) L.dst_row[i] += s_rb[q];
+  }
+  const int n = R * d.nsub;
+  for (int64_t t = i0; t < N; t += stride) {
+    const int c = L.shared_rank[t];
+    const int r = (int)t / d.T, tt = (int)t - r * d.T;
+    L.shared_row[t] += s_sb[c] + s.wsub_cnt[(int64_t)c * n + r * d.nsub + tt / kPlanSubT];
+  }
+}
+
 // Standalone Waterfill: one thread per token; the waterline is recomputed per
 // block from the loads (R <= 128 values).
 __global__ void __launch_bounds__(256)
@@ -1173,8 +1223,7 @@ cudaError_t set_plan_attributes(int max_smem) {
   if ((e = allow_solve<8>(max_smem)) != cudaSuccess) return e;
   if ((e = allow_max_dynamic_smem(k_hist, max_smem)) != cudaSuccess) return e;
   if ((e = allow_max_dynamic_smem(k_assign<0>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_assign<1>, max_smem)) != cudaSuccess) return e;
-  return allow_max_dynamic_smem(k_assign<2>, max_smem);
+  return allow_max_dynamic_smem(k_assign<1>, max_smem);
 }
 
 template <int SMAX>
@@ -1225,7 +1274,11 @@ cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, c
     if (err != cudaSuccess) return err;
     err = launch_pdl(k_shared_scan, (unsigned)d.R, kScanThreads, 0, st, d, L, s);
     if (err != cudaSuccess) return err;
-    if (nblk > 0) err = launch_pdl(k_assign<2>, nblk, bt, assign_smem(d, 2), st, ids, d, L, s);
+    const int64_t A4 = (int64_t)d.R * d.T * d.K / 4, N = (int64_t)d.R * d.T;
+    const int64_t work = A4 > N ? A4 : N;
+    const int64_t fblk = (work + kFixThreads - 1) / kFixThreads;
+    if (work > 0)
+      err = launch_pdl(k_fixup, (unsigned)(fblk < 2048 ? fblk : 2048), kFixThreads, 0, st, d, L, s);
   }
   if (err != cudaSuccess) return err;
   return cudaGetLastError();

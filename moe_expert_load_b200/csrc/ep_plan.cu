@@ -527,31 +527,52 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   int32_t* iloc = s_iloc[warp];
   int32_t* jof = s_jof[warp];
 
+  // the load column of e: independent of the instance lookups below, so its
+  // loads are issued first
+  int lcol[kRW];
+#pragma unroll
+  for (int k = 0; k < kRW; ++k) {
+    const int r = lane + 32 * k;
+    lcol[k] = r < R ? L.load[r * E + e] : 0;
+  }
   const int h = home_of(e, E, R);
   const int hcol = e - nat_first(h, E, R);
-  const int p0 = L.rep_eptr[e], nrep = L.rep_eptr[e + 1] - p0;
-  const int ninst = nrep + 1;
-  // position of the native among the instances (replicas are in rank order)
-  int np = 0;
-  for (int j = lane; j < nrep; j += 32) np += (L.rep_list[p0 + j] / S) < h;
-  np = __reduce_add_sync(kFull, np);
+  const int nat_rel = s.inst_rel[h * G + hcol], nat_q = L.inst_quota[h * G + hcol];
   for (int q = lane; q < R; q += 32) jof[q] = -1;
   __syncwarp();
-  for (int j = lane; j < ninst; j += 32) {
-    int rank, col;
-    if (j == np) {
-      rank = h;
-      col = hcol;
-    } else {
-      const int slot = L.rep_list[p0 + (j < np ? j : j - 1)];
-      rank = slot / S;
-      col = d.Gmax + (slot - rank * S);
+  // instances in instance order: the replica slots holding e (scanned in slot
+  // order, i.e. rank order; none is on the home rank h) with the native placed
+  // after the replicas on ranks below h.  Every slot's entries are loaded in
+  // one round, independent of each other.
+  int nrep = 0, np = 0;
+  for (int i0 = 0; i0 < R * S; i0 += 32) {
+    const int i = i0 + lane;
+    const int q = i / S, col = d.Gmax + (i - (i / S) * S);
+    bool hit = false;
+    int rel = 0, quota = 0;
+    if (i < R * S) {
+      hit = L.inst_expert[q * G + col] == e;
+      rel = s.inst_rel[q * G + col];
+      quota = L.inst_quota[q * G + col];
     }
-    irank[j] = rank;
-    irel[j] = s.inst_rel[rank * G + col];
-    iq[j] = L.inst_quota[rank * G + col];
-    jof[rank] = j;
+    const unsigned m = __ballot_sync(kFull, hit);
+    if (hit) {
+      const int j = nrep + __popc(m & lanemask_lt()) + (q > h ? 1 : 0);
+      irank[j] = q;
+      irel[j] = rel;
+      iq[j] = quota;
+      jof[q] = j;
+    }
+    nrep += __popc(m);
+    np += __popc(__ballot_sync(kFull, hit && q < h));
   }
+  if (lane == 0) {
+    irank[np] = h;
+    irel[np] = nat_rel;
+    iq[np] = nat_q;
+    jof[h] = np;
+  }
+  const int ninst = nrep + 1;
   __syncwarp();
   // local take and residual demand of every source rank (lane owns r = lane + 32k)
   int Dr[kRW], locr[kRW];
@@ -561,7 +582,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
     Dr[k] = 0;
     locr[k] = 0;
     if (r < R) {
-      const int l = L.load[r * E + e];
+      const int l = lcol[k];
       const int j = jof[r];
       const int loc = j >= 0 ? min(l, iq[j]) : 0;
       locr[k] = loc;

@@ -206,10 +206,17 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   }
   __syncthreads();
   if (warp == 0) {
-    int a = 0;
-    for (int q = lane; q < R; q += 32) a += s_W0[q];
+    int a = 0, bm = 0;
+    for (int q = lane; q < R; q += 32) {
+      a += s_W0[q];
+      bm = max(bm, s_W0[q]);
+    }
     a = __reduce_add_sync(kFull, a);
-    if (lane == 0) s_A = a;
+    bm = (int)__reduce_max_sync(kFull, (unsigned)bm);
+    if (lane == 0) {
+      s_A = a;
+      L.stats->before_max = bm;
+    }
   }
   __syncthreads();
   const int A = s_A;
@@ -460,11 +467,6 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     }
     for (int q = tid; q < R; q += nthr) s.slack[q] = (int)max(H - (int64_t)s_Wf[q], (int64_t)0);
   }
-  if (tid == 0) {
-    int bm = 0;
-    for (int q = 0; q < R; ++q) bm = max(bm, s_W0[q]);
-    L.stats->before_max = bm;
-  }
   // replica lists grouped by expert (CSR), instance order inside an expert
   if (warp == 0) {
     int carry = 0, ncarry = 0;
@@ -488,14 +490,20 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       ncarry += __shfl_sync(kFull, fincl, 31);
     }
     if (lane == 0) L.rep_nexp[0] = ncarry;
-  }
-  __syncthreads();
-  for (int i = tid; i < R * S; i += nthr) {
-    const int e = s_se[i];
-    if (e < 0) continue;
-    int before = 0;
-    for (int i2 = 0; i2 < i; ++i2) before += (s_se[i2] == e);
-    L.rep_list[s_eptr[e] + before] = i;
+    // each filled slot's place in its expert's list: the list's start plus
+    // the earlier slots of that expert (32 slots at a time, in slot order)
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) cnt_e[e] = s_eptr[e];
+    __syncwarp();
+    for (int i0 = 0; i0 < R * S; i0 += 32) {
+      const int i = i0 + lane;
+      const int e = i < R * S ? s_se[i] : -1;
+      const unsigned peers = __match_any_sync(kFull, e);
+      if (e >= 0) L.rep_list[cnt_e[e] + __popc(peers & lanemask_lt())] = i;
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) cnt_e[e] += __popc(peers);
+      __syncwarp();
+    }
   }
 }
 

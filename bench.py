@@ -198,8 +198,8 @@ E2E_CHUNKS = 8  # token chunks of the end-to-end step's hidden-state copy
 
 
 def _balance_launches(w):
-    # clear, hist, solve, reroute + assign (or assign, shared scan, assign)
-    return 4 + (3 if w.shared_expert else 1)
+    # hist, solve, reroute + assign (or assign, shared scan, fix-up)
+    return 3 + (3 if w.shared_expert else 1)
 
 
 def _ratio(st, R):

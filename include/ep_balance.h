@@ -170,6 +170,10 @@ EP_API void ep_plan_destroy(ep_plan* plan);
  * solve replica placement and per-instance quotas, reroute local-first, and
  * assign every (token, k) its dispatch row, all into the layer's slot of the
  * plan cache (overwriting it).  Every rank would compute this identically.
+ * Calls on one plan share its scratch: they must not overlap on the GPU (one
+ * stream, or streams ordered by events).  The first call of a plan zeroes the
+ * scratch accumulators with one cudaMemsetAsync on `stream`; a call whose
+ * launch fails (EP_ERR_CUDA) makes the next call zero them again.
  */
 EP_API ep_status_t ep_balance_layer(ep_plan* plan, int32_t layer, const int32_t* d_topk_ids,
                              void* stream);

@@ -24,11 +24,11 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
   // per layer (offset inside one layer block)
   size_t load, expert_total, W0, W, inst_expert, inst_quota, inst_off, rank_base, dst_row,
-      shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, stats, tickets;
+      shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, stats;
   size_t layer_bytes;
   // scratch (absolute)
   size_t sub_cnt, blk_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase,
-      shared_tot, asg_rank;
+      shared_tot, asg_rank, acc_load, acc_tot, acc_misc;
   size_t scratch_bytes;
   size_t total;
 };
@@ -87,11 +87,9 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   Layout L{};
   const size_t i4 = sizeof(int32_t);
   Bump b;
-  // stats, load, expert_total and tickets are contiguous: one memset clears them
   L.stats = b.take(sizeof(ep_layer_stats));
   L.load = b.take(i4 * d.R * d.E);
   L.expert_total = b.take(i4 * d.E);
-  L.tickets = b.take(i4 * 4);
   L.W0 = b.take(i4 * d.R);
   L.W = b.take(i4 * d.R);
   L.inst_expert = b.take(i4 * d.R * d.G);
@@ -122,6 +120,10 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.sbase = s.take(i4 * d.R);
   L.shared_tot = s.take(i4 * d.R);
   L.asg_rank = s.take(d.sh ? (size_t)d.R * d.T * d.K : 0);
+  // contiguous: zeroed together once, before the plan's first balance call
+  L.acc_load = s.take(i4 * (size_t)d.R * d.E);
+  L.acc_tot = s.take(i4 * d.E);
+  L.acc_misc = s.take(i4 * 4);
   L.total = s.off;
   L.scratch_bytes = s.off - L.layer_bytes * (size_t)num_layers;
   return L;
@@ -140,6 +142,7 @@ struct ep_plan {
   int device;
   int num_sms;
   unsigned char* planned;  // per layer: balanced at least once
+  bool acc_zero;           // the scratch accumulators are known to be zero
 };
 
 namespace {
@@ -152,7 +155,6 @@ ep::LayerBuf layer_buf(const ep_plan* p, int layer) {
   ep::LayerBuf L;
   L.load = at(p, b + l.load);
   L.expert_total = at(p, b + l.expert_total);
-  L.tickets = at(p, b + l.tickets);
   L.W0 = at(p, b + l.W0);
   L.W = at(p, b + l.W);
   L.inst_expert = at(p, b + l.inst_expert);
@@ -187,6 +189,9 @@ ep::Scratch scratch(const ep_plan* p) {
   s.sbase = at(p, l.sbase);
   s.shared_tot = at(p, l.shared_tot);
   s.asg_rank = p->d.sh ? reinterpret_cast<uint8_t*>(p->ws + l.asg_rank) : nullptr;
+  s.acc_load = at(p, l.acc_load);
+  s.acc_tot = at(p, l.acc_tot);
+  s.acc_misc = at(p, l.acc_misc);
   return s;
 }
 
@@ -260,6 +265,7 @@ ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t works
   p->ws_bytes = workspace_bytes;
   p->device = dev;
   p->num_sms = sms;
+  p->acc_zero = false;
   *out = p;
   return EP_OK;
 }
@@ -275,9 +281,19 @@ ep_status_t ep_balance_layer(ep_plan* plan, int32_t layer, const int32_t* d_topk
   ep_status_t st = check_layer(plan, layer);
   if (st != EP_OK) return st;
   if (!d_topk_ids && plan->d.T > 0) return EP_ERR_INVALID_ARGUMENT;
-  st = cuda_status(ep::launch_balance(plan->d, layer_buf(plan, layer), scratch(plan), d_topk_ids,
-                                      static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!plan->acc_zero) {
+    // the workspace arrives uninitialised; after this every balance call
+    // leaves the accumulators zero for the next
+    const Layout& l = plan->lay;
+    const size_t bytes = l.acc_misc + 4 * sizeof(int32_t) - l.acc_load;
+    st = cuda_status(cudaMemsetAsync(plan->ws + l.acc_load, 0, bytes, s));
+    if (st != EP_OK) return st;
+    plan->acc_zero = true;
+  }
+  st = cuda_status(ep::launch_balance(plan->d, layer_buf(plan, layer), scratch(plan), d_topk_ids, s));
   if (st == EP_OK) plan->planned[layer] = 1;
+  else plan->acc_zero = false;  // a partly launched chain may leave them non-zero
   return st;
 }
 

@@ -38,7 +38,6 @@ struct Dims {
 struct LayerBuf {
   int32_t* load;          // [R][E]
   int32_t* expert_total;  // [E]
-  int32_t* tickets;       // [4] arrival counters, zeroed with stats/load/expert_total
   int32_t* W0;            // [R]
   int32_t* W;             // [R]
   int32_t* inst_expert;   // [R][G]
@@ -71,6 +70,12 @@ struct Scratch {
   int32_t* sbase;     // [R] first row of each rank's shared column
   int32_t* shared_tot;  // [R] shared-slot rows per destination rank
   uint8_t* asg_rank;    // [R][T][K] destination rank of each assignment (shared expert only)
+  // Accumulators that are zero whenever no balance call is running: the
+  // histogram adds into them, the solve and the rerouting copy them out to the
+  // layer and zero them again, and the arrival ticket resets itself.
+  int32_t* acc_load;    // [R][E]
+  int32_t* acc_tot;     // [E]
+  int32_t* acc_misc;    // [0] status bits of the histogram, [1] arrival ticket
 };
 
 // ---- native placement: contiguous balanced blocks ---------------------------

@@ -54,13 +54,14 @@ constexpr int kAsgBatch = 8;   // ids per lane per pass in k_assign
 // sub-chunk at once (at most 16 ids per lane) and counts it into a private
 // shared-memory histogram with shared atomic adds; the warp writes its row of
 // counts and the block writes the sum of its rows (the two levels of bases of
-// the stable ordinals, used by k_assign).  After the predecessor (the kernel
-// that clears the layer's counters) has finished, the block adds its sum to the
-// load matrix L[r][e] and the expert totals with integer atomics
-// (order-independent, so the result is deterministic).
+// the stable ordinals, used by k_assign).  The block then adds its sum to the
+// load-matrix and expert-total accumulators with integer atomics
+// (order-independent, so the result is deterministic); they are zero on entry
+// and the solve and the rerouting move them into the layer.  The first kernel
+// of the plan: a plain launch, so the ids are complete when it starts.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, 6)
-k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, LayerBuf L) {
+k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
   extern __shared__ int32_t sm_hist[];
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,26 +106,17 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s, LayerBuf L) {
       blk[e] = csum[u];
     }
   }
-  pdl_wait();  // the layer's counters and status word have been cleared
-  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&L.stats->status, EP_DEV_BAD_ID);
+  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&s.acc_misc[0], EP_DEV_BAD_ID);
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int e = threadIdx.x + u * blockDim.x;
     if (e < E && csum[u]) {
-      atomicAdd(&L.load[r * E + e], csum[u]);
-      atomicAdd(&L.expert_total[e], csum[u]);
+      atomicAdd(&s.acc_load[r * E + e], csum[u]);
+      atomicAdd(&s.acc_tot[e], csum[u]);
     }
   }
 }
 
-// Clears the layer's stats, load matrix, expert totals and arrival tickets
-// (adjacent in the layer block) before the histogram adds into them.
-__global__ void __launch_bounds__(256) k_clear_layer(int4* __restrict__ p, int64_t n16) {
-  pdl_trigger();
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16;
-       i += (int64_t)gridDim.x * blockDim.x)
-    p[i] = make_int4(0, 0, 0, 0);
-}
 
 // Warp argmax over the ranks lane + 32k (k < RW) with ok[k] set: the largest
 // v, smallest rank on ties.  When every v is below 2^24 the value and the rank
@@ -194,8 +186,18 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
 
   pdl_trigger();
   pdl_wait();
-  for (int e = tid; e < E; e += nthr) Tot[e] = L.expert_total[e];
-  if (tid == 0) s_iter_cap_hit = 0;
+  for (int e = tid; e < E; e += nthr) {
+    const int v = s.acc_tot[e];
+    Tot[e] = v;
+    L.expert_total[e] = v;
+    s.acc_tot[e] = 0;  // zero again for the next call
+  }
+  if (tid == 0) {
+    s_iter_cap_hit = 0;
+    L.stats->status = s.acc_misc[0];  // the first status bits of this call
+    L.stats->reserved0 = 0;
+    s.acc_misc[0] = 0;
+  }
   __syncthreads();
   if (tid < R) {
     const int f = tid * eb + min(tid, er), n = eb + (tid < er ? 1 : 0);
@@ -541,7 +543,13 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
 #pragma unroll
   for (int k = 0; k < kRW; ++k) {
     const int r = lane + 32 * k;
-    lcol[k] = r < R ? L.load[r * E + e] : 0;
+    if (r < R) {
+      lcol[k] = s.acc_load[r * E + e];
+      L.load[r * E + e] = lcol[k];
+      s.acc_load[r * E + e] = 0;  // zero again for the next call
+    } else {
+      lcol[k] = 0;
+    }
   }
   const int h = home_of(e, E, R);
   const int hcol = e - nat_first(h, E, R);
@@ -1073,11 +1081,12 @@ __global__ void __launch_bounds__(kScanThreads) k_shared_scan(Dims d, LayerBuf L
   if (tid == 0) {
     s.shared_tot[c] = s_carry;
     __threadfence();
-    s_last = atomicAdd(&L.tickets[0], 1) == R - 1;
+    s_last = atomicAdd(&s.acc_misc[1], 1) == R - 1;
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (tid == 0) s.acc_misc[1] = 0;  // every block has arrived: reset for the next call
   if (warp == 0) {
     int carry = 0;
     for (int q0 = 0; q0 < R; q0 += 32) {
@@ -1275,20 +1284,14 @@ cudaError_t launch_solve(const Dims& d, const LayerBuf& L, const Scratch& s, cud
 
 cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, const int32_t* ids,
                            cudaStream_t st) {
-  // stats, load matrix, expert totals and tickets are adjacent in the layer
-  // block (256-byte aligned pieces): one clearing kernel covers them
-  const size_t zero_bytes = reinterpret_cast<const char*>(L.tickets + 4) -
-                            reinterpret_cast<const char*>(L.stats);
-  const int64_t n16 = (int64_t)((zero_bytes + 15) / 16);
-  const int64_t cblocks = (n16 + 255) / 256;
-  k_clear_layer<<<(unsigned)(cblocks < 64 ? cblocks : 64), 256, 0, st>>>(
-      reinterpret_cast<int4*>(L.stats), n16);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+  // the histogram is a plain launch (it reads the caller's ids at once); every
+  // later kernel is a programmatic dependent launch of its predecessor
+  cudaError_t err = cudaSuccess;
   const unsigned nblk = (unsigned)(d.R * ((d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock));
   const unsigned bt = kWarpsPerBlock * 32;
   if (nblk > 0) {
-    err = launch_pdl(k_hist, nblk, bt, hist_smem(d), st, ids, d, s, L);
+    k_hist<<<nblk, bt, hist_smem(d), st>>>(ids, d, s);
+    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
   err = launch_solve(d, L, s, st);

@@ -87,6 +87,29 @@ def test_plan_parity_bad_ids_and_ragged_tail():
     assert g["dst_row"][0, 3, 1] == -1
 
 
+@pytest.mark.parametrize("shared", [False, True])
+def test_plan_state_does_not_carry_between_calls(shared):
+    # one plan, one layer, several calls in a row with different ids (one with
+    # bad ids, one empty-looking skew, then the first again): every call must
+    # equal the oracle on its own ids, and a status bit of one call must not
+    # survive into the next
+    base = get_config("tiny").replace(T=1000, shared_expert=shared)
+    rng = np.random.default_rng(11)
+    good = topk_ids(get_config("tiny"))[:, :1000].copy()
+    bad = good.copy()
+    bad[1, 5, 0] = base.E + 3
+    skew = np.zeros_like(good)
+    skew[..., 1] = 1
+    shuffled = rng.permutation(good.reshape(-1)).reshape(good.shape).astype(np.int32)
+    plan = Plan(config_from_workload(base, num_layers=2))
+    for ids in (good, bad, skew, shuffled, good):
+        for layer in (0, 1):
+            gpu_plan(base, ids, plan=plan, layer=layer)
+            g = fetch(plan, layer)
+            compare_plan(g, oracle_plan(base, ids), base)
+            assert (g["stats"]["status"] & 1) == (1 if ids is bad else 0)
+
+
 def test_plan_deterministic():
     w = get_config("dsv3")
     ids = topk_ids(w)

@@ -21,6 +21,8 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kWarpsPerBlock = kPlanWarps;
+// experts per thread when a block of the plan kernels covers all E <= kMaxE
+constexpr int kExpPerThread = kMaxE / (kWarpsPerBlock * 32);
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -95,9 +97,9 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
   }
   __syncthreads();
   int32_t* blk = s.blk_cnt + ((int64_t)r * nbpr + b) * E;
-  int csum[4];
+  int csum[kExpPerThread];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < kExpPerThread; ++u) {
     const int e = threadIdx.x + u * blockDim.x;
     csum[u] = 0;
     if (e < E) {
@@ -108,7 +110,7 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
   }
   if (__any_sync(kFull, bad) && lane == 0) atomicOr(&s.acc_misc[0], EP_DEV_BAD_ID);
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < kExpPerThread; ++u) {
     const int e = threadIdx.x + u * blockDim.x;
     if (e < E && csum[u]) {
       atomicAdd(&s.acc_load[r * E + e], csum[u]);
@@ -854,9 +856,9 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   {
     const int per = (E + nthr - 1) / nthr;
     const int eb = tid * per;
-    int cnt[4], s0[4], local = 0;
+    int cnt[kExpPerThread], s0[kExpPerThread], local = 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kExpPerThread; ++u) {
       const int e = eb + u;
       cnt[u] = 0;
       s0[u] = 0;
@@ -879,7 +881,7 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     for (int w = 0; w < warp; ++w) off += s_wsum[w];
     if (tid == nthr - 1) s_total = off + local;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kExpPerThread; ++u) {
       const int e = eb + u;
       if (u < per && e < E) {
         const int64_t gb = (int64_t)e * 3 * R + s0[u];

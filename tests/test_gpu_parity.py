@@ -38,6 +38,78 @@ def test_plan_parity_large_counts():
     assert o.replicas > 0
 
 
+def _skewed_topk(rng, R, T, E, K, zipf_s):
+    """Distinct top-K ids per token from a Zipf-skewed popularity (Gumbel top-k)."""
+    logp = -zipf_s * np.log(np.arange(1, E + 1, dtype=np.float64))
+    logp = logp[rng.permutation(E)]
+    g = rng.gumbel(size=(R * T, E)) + logp
+    ids = np.argpartition(-g, K - 1, axis=1)[:, :K]
+    return ids.reshape(R, T, K).astype(np.int32)
+
+
+@pytest.mark.parametrize("R,E,K,T,S,m,shared", [
+    (128, 1024, 16, 96, 8, 1, False),   # every limit at once: 4 rank words, 8 slots, 8 natives
+    (128, 1024, 16, 96, 8, 16, True),
+    (128, 128, 16, 200, 8, 4, True),    # one native per rank
+    (32, 1024, 8, 300, 2, 8, False),    # 32 natives per rank (the solver's lane limit)
+    (1, 32, 16, 500, 8, 1, True),       # a single rank
+])
+def test_plan_parity_maximum_shapes(R, E, K, T, S, m, shared):
+    rng = np.random.default_rng(R * 7919 + E + K + S)
+    ids = _skewed_topk(rng, R, T, E, K, 1.3)
+    w = get_config("tiny").replace(R=R, E=E, K=K, T=T, S=S, m=m, J=16, shared_expert=shared)
+    o = oracle_plan(w, ids)
+    compare_plan(fetch(gpu_plan(w, ids)), o, w)
+
+
+@pytest.mark.parametrize("K,T,m,shared", [(8, 600, 1, False), (16, 300, 4, True)])
+def test_plan_parity_every_slot_filled(K, T, m, shared):
+    # rank 0's 32 natives (the solver's lane limit) carry all the load, so the
+    # greedy moves whole experts until each of the 3 other ranks holds 8
+    # replicas (every slot of the 8-slot layout in use)
+    R, E, S = 4, 128, 8
+    rng = np.random.default_rng(5)
+    logp = np.full(E, -8.0)
+    logp[:32] = 0.0
+    g = rng.gumbel(size=(R * T, E)) + logp
+    ids = np.argpartition(-g, K - 1, axis=1)[:, :K].reshape(R, T, K).astype(np.int32)
+    w = get_config("tiny").replace(R=R, E=E, K=K, T=T, S=S, m=m, J=16, shared_expert=shared)
+    o = oracle_plan(w, ids)
+    assert (o.inst_expert[1:, o.Gmax:o.Gmax + S] >= 0).all()
+    compare_plan(fetch(gpu_plan(w, ids)), o, w)
+
+
+def test_stage_and_reduce_every_slot_filled():
+    # the 24-replica plan above: staging copies each filled slot's expert, the
+    # reduction adds up to 3 replicas per expert in instance order
+    R, E, S, K, T, Wn = 4, 128, 8, 8, 600, 1000
+    rng = np.random.default_rng(5)
+    logp = np.full(E, -8.0)
+    logp[:32] = 0.0
+    g = rng.gumbel(size=(R * T, E)) + logp
+    ids = np.argpartition(-g, K - 1, axis=1)[:, :K].reshape(R, T, K).astype(np.int32)
+    w = get_config("tiny").replace(R=R, E=E, K=K, T=T, S=S, m=1, J=16)
+    plan = gpu_plan(w, ids, expert_weight_elems=Wn)
+    o = oracle_plan(w, ids)
+    native = torch.from_numpy(rng.integers(-30000, 30000, (E, Wn)).astype(np.int16)).cuda()
+    slots = torch.full((R, S, Wn), 3, dtype=torch.int16, device="cuda")
+    plan.stage_replicas(0, native.view(torch.bfloat16), slots.view(torch.bfloat16))
+    g32 = (rng.standard_normal((R, S, Wn)) * 1e-2).astype(np.float32)
+    g_np = (g32.view(np.uint32) >> 16).astype(np.uint16)
+    g_t = torch.from_numpy(g_np.view(np.int16)).cuda().view(torch.bfloat16)
+    nat_np = rng.standard_normal((E, Wn)).astype(np.float32)
+    nat_t = torch.from_numpy(nat_np).cuda()
+    plan.reduce_replica_grads(0, g_t, nat_t)
+    torch.cuda.synchronize()
+    want_slots = np.full((R, S, Wn), 3, np.int16)
+    oracle.stage(o, native.cpu().numpy(), want_slots)
+    np.testing.assert_array_equal(slots.cpu().numpy(), want_slots)
+    want_nat, want_g = nat_np.copy(), g_np.copy()
+    oracle.reduce_grads(o, want_g, want_nat)
+    np.testing.assert_array_equal(nat_t.cpu().numpy().view(np.uint32), want_nat.view(np.uint32))
+    np.testing.assert_array_equal(g_t.view(torch.int16).cpu().numpy().view(np.uint16), want_g)
+
+
 def test_plan_parity_sweep_layers_cached():
     w = get_config("sweep")
     layers = [0, 1, 3, 47, 93]

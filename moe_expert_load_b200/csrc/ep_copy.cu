@@ -1,5 +1,6 @@
 // HBM-bound data movement for sm_100a: dispatch permutation of hidden rows,
-// replica weight staging into the shared slots, replica gradient reduction.
+// its reverse (the gate-weighted combine), replica weight staging into the
+// shared slots, replica gradient reduction.
 //
 // Dispatch (UltraEP page, "300 µs to level MoE expert load": token dispatch
 // starts once replicas are in place; Waterfill page §"Shared expert fusion":
@@ -25,7 +26,7 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // ---------------------------------------------------------------------------
 // a6: dispatch permutation.  One warp per token at a time (grid-stride over
-// tokens): lanes 0..K-1 fetch the token's K dispatch rows, lane K its
+// the tokens [n0, N) of the call): lanes 0..K-1 fetch the token's K dispatch rows, lane K its
 // shared-slot row, keeping those inside the destination-rank window
 // [row_lo, row_hi); the warp loads the bf16 row once into registers (16-byte
 // vector loads, up to 8 KiB per pass) and stores it to every kept row with

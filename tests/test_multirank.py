@@ -79,3 +79,13 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     line = bench.run_reference(Args())
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["cores"] == 1
+
+
+def test_traffic_record_hash_ignores_comments(tmp_path):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    code = "int a; // note\n/* block\n comment */ int b;\n\n  // only a comment\nint c;\n"
+    assert bench._code_only(code) == "int a;\n int b;\nint c;"
+    assert bench._code_only(code.replace("note", "other note")) == bench._code_only(code)
+    assert bench._code_only(code.replace("int c", "int d")) != bench._code_only(code)

@@ -297,6 +297,20 @@ def run_gpu(args):
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
     plan_us = sorted(1e3 * t for t in _timed(torch, lambda: plan.balance_layer(0, ids),
                                              args.plan_iters, stream, flush, skip=3))
+    # the same call replayed from a CUDA graph (the chain captured once)
+    try:
+        gstream = torch.cuda.Stream(device=dev)
+        gstream.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gstream):
+            plan.balance_layer(0, ids)
+        stream.wait_stream(gstream)
+        us = sorted(1e3 * t for t in _timed(torch, graph.replay, args.plan_iters, stream, flush,
+                                            skip=3))
+        plan_graph = {"median": _median(us), "mean": sum(us) / len(us), "iters": len(us)}
+        del graph
+    except RuntimeError as err:  # reported, not fatal: the eager figure stands
+        plan_graph = {"error": str(err).splitlines()[0]}
     stage_ms = _median(_timed(torch, lambda: plan.stage_replicas(0, native_w, slots), 5, stream, flush))
     reduce_ms = _median(_timed(torch, lambda: plan.reduce_replica_grads(0, slot_grads, native_grads),
                                5, stream, flush))
@@ -403,6 +417,7 @@ def run_gpu(args):
         # mean over the iterations resolves finer than the median
         "plan_us": {"median": _median(plan_us), "mean": sum(plan_us) / len(plan_us),
                     "p90": plan_us[int(len(plan_us) * 0.9)], "iters": len(plan_us)},
+        "plan_us_cuda_graph": plan_graph,
         "permute_gbs": achieved,
         "stage_gbs": stage_bytes / (stage_ms * 1e-3) / 1e9 if n_rep else 0.0,
         "reduce_gbs": reduce_bytes / (reduce_ms * 1e-3) / 1e9 if n_rep else 0.0,

@@ -305,6 +305,35 @@ def test_dispatch_tokens_argument_errors():
     assert plan.read_layer_stats(0)["status"] == 0
 
 
+def test_balance_and_dispatch_replay_from_cuda_graph():
+    # the plan chain (programmatic dependent launches) and the dispatch,
+    # captured once and replayed on new ids written into the same buffer
+    w = get_config("tiny").replace(T=1000, shared_expert=True)
+    base = topk_ids(get_config("tiny"))[:, :1000].copy()
+    rng = np.random.default_rng(3)
+    sets = [base, rng.permutation(base.reshape(-1)).reshape(base.shape).astype(np.int32),
+            np.ascontiguousarray(base[:, ::-1])]
+    plan = Plan(config_from_workload(w))
+    ids_buf = torch.from_numpy(sets[1]).cuda()
+    hidden = _hidden(w, 4)
+    out = torch.zeros((w.A + w.N, w.hidden), dtype=torch.bfloat16, device="cuda")
+    plan.balance_layer(0, ids_buf)  # outside the graph: the plan's first call
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        plan.balance_layer(0, ids_buf)
+        plan.dispatch_layout(0, hidden, out=out)
+    for ids in sets:
+        ids_buf.copy_(torch.from_numpy(ids))
+        graph.replay()
+        torch.cuda.synchronize()
+        o = oracle_plan(w, ids)
+        compare_plan(fetch(plan), o, w)
+        want = oracle.permute(o, hidden.view(torch.int16).cpu().numpy())
+        np.testing.assert_array_equal(out.view(torch.int16).cpu().numpy()[: o.rows], want)
+    del graph
+
+
 def test_dispatch_capacity_overflow_is_flagged_not_written():
     w = get_config("tiny")
     ids = topk_ids(w)

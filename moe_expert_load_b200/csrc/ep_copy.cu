@@ -9,8 +9,8 @@
 // communication kernels": a persistent kernel pulls fixed-size tiles from a
 // device-side task list) are whole-row / whole-tile bit copies in which each
 // source byte is read from HBM once and written once per destination: a warp
-// stages up to 8 KiB in registers with 16-byte vector loads and stores it to
-// every destination with 16-byte vector stores.  See k_permute for the
+// stages a slice of the row (or tile) in registers with vector loads and
+// stores it to every destination with vector stores.  See k_permute for the
 // measurements that chose this over bulk-copy (TMA) staging through shared
 // memory.  Nothing here waits on another thread, block or device.
 #include <cuda_bf16.h>
@@ -28,12 +28,14 @@ constexpr unsigned kFull = 0xffffffffu;
 // a6: dispatch permutation.  One warp per token at a time (grid-stride over
 // the tokens [n0, N) of the call): lanes 0..K-1 fetch the token's K dispatch rows, lane K its
 // shared-slot row, keeping those inside the destination-rank window
-// [row_lo, row_hi); the warp loads the bf16 row once into registers (16-byte
-// vector loads, up to 8 KiB per pass) and stores it to every kept row with
-// 16-byte vector stores.  Tokens with no row in the window are not read.
+// [row_lo, row_hi); the warp loads the bf16 row once into registers (32-byte
+// vector loads, 4 KiB per pass, where the row size and both buffers are
+// 32-byte aligned; else 16-byte loads, 8 KiB per pass) and stores it to every
+// kept row with vector stores of the same width.  Tokens with no row in the
+// window are not read.
 //
 // Measured on B200 (qwen, 19.3 GB per launch): this register-staged form moves
-// 6.1-6.2 TB/s; the same copy with bulk-copy (TMA) loads into shared memory
+// 6.1-6.2 TB/s with 16-byte vectors; the same copy with bulk-copy (TMA) loads into shared memory
 // and bulk stores stayed at 5.6-5.7 TB/s for every stage count (2-8) and
 // occupancy tried, and TMA loads with vector stores from shared memory at
 // 5.3-5.5 TB/s, so the bulk-copy engine is not used for this 1:K fan-out.
@@ -53,14 +55,48 @@ struct PermuteArgs {
 };
 
 constexpr int kPermuteThreads = 128;
-constexpr int kRowWordsPerLane = 16;  // 16 x 16 B per lane = 8 KiB per warp pass
 
+// 32-byte vectors (ld/st.global.v8.b32, sm_100): rows and both buffers must be
+// 32-byte aligned.
+struct Vec32 {
+  uint32_t x[8];
+};
+__device__ __forceinline__ Vec32 load32(const Vec32* p) {
+  Vec32 v;
+  asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v.x[0]), "=r"(v.x[1]), "=r"(v.x[2]), "=r"(v.x[3]), "=r"(v.x[4]),
+                 "=r"(v.x[5]), "=r"(v.x[6]), "=r"(v.x[7])
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void store32(Vec32* p, const Vec32& v) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.x[0]),
+               "r"(v.x[1]), "r"(v.x[2]), "r"(v.x[3]), "r"(v.x[4]), "r"(v.x[5]), "r"(v.x[6]),
+               "r"(v.x[7])
+               : "memory");
+}
+__device__ __forceinline__ uint4 load32(const uint4* p) { return *p; }
+__device__ __forceinline__ void store32(uint4* p, const uint4& v) { *p = v; }
+
+// Words per lane per pass: 4 x 32 B (4 KiB per warp pass) with 32-byte
+// vectors, 16 x 16 B (8 KiB) otherwise.  Measured on the qwen / dsv3 layers:
+// 6.28-6.30 / 6.22-6.25 TB/s with 4 x 32 B, 6.13 / 6.09 with 16 x 16 B, 5.7 /
+// 5.6 with 8 x 32 B (114 registers, lower occupancy).
+template <typename W>
+struct PermuteShape {
+  static constexpr int kWordsPerLane = sizeof(W) == 32 ? 4 : 16;
+};
+
+template <typename W>
 __global__ void __launch_bounds__(kPermuteThreads) k_permute(PermuteArgs a) {
+  constexpr int kWPL = PermuteShape<W>::kWordsPerLane;
   const int lane = threadIdx.x & 31;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int row_lo = a.rank_base[a.rank_begin];
   const int row_hi = a.rank_base[a.rank_end];
-  const int row16 = a.row16;
+  const int roww = a.row16 * 16 / (int)sizeof(W);  // words of W per row
+  const W* hidden = reinterpret_cast<const W*>(a.hidden);
+  W* out = reinterpret_cast<W*>(a.out);
   bool overflow = false;
   for (int64_t n = a.n0 + (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); n < a.N; n += nw) {
     int d = -1;
@@ -73,23 +109,23 @@ __global__ void __launch_bounds__(kPermuteThreads) k_permute(PermuteArgs a) {
     }
     const unsigned m = __ballot_sync(kFull, d >= 0);
     if (!m) continue;
-    const uint4* src = a.hidden + n * row16;
-    for (int c0 = 0; c0 < row16; c0 += kRowWordsPerLane * 32) {
-      uint4 v[kRowWordsPerLane];
+    const W* src = hidden + n * roww;
+    for (int c0 = 0; c0 < roww; c0 += kWPL * 32) {
+      W v[kWPL];
 #pragma unroll
-      for (int k = 0; k < kRowWordsPerLane; ++k) {
+      for (int k = 0; k < kWPL; ++k) {
         const int idx = c0 + k * 32 + lane;
-        if (idx < row16) v[k] = src[idx];
+        if (idx < roww) v[k] = load32(src + idx);
       }
       unsigned mm = m;
       while (mm) {
         const int from = __ffs(mm) - 1;
         mm &= mm - 1;
-        uint4* dst = a.out + (int64_t)__shfl_sync(kFull, d, from) * row16;
+        W* dst = out + (int64_t)__shfl_sync(kFull, d, from) * roww;
 #pragma unroll
-        for (int k = 0; k < kRowWordsPerLane; ++k) {
+        for (int k = 0; k < kWPL; ++k) {
           const int idx = c0 + k * 32 + lane;
-          if (idx < row16) dst[idx] = v[k];
+          if (idx < roww) store32(dst + idx, v[k]);
         }
       }
     }
@@ -437,7 +473,12 @@ cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden
   const int64_t warps = (a.N - a.n0);
   const int64_t blocks = (warps + kPermuteThreads / 32 - 1) / (kPermuteThreads / 32);
   const int64_t grid = blocks < (int64_t)num_sms * 12 ? blocks : (int64_t)num_sms * 12;
-  k_permute<<<(unsigned)grid, kPermuteThreads, 0, st>>>(a);
+  const bool w32 = a.row16 % 2 == 0 && (reinterpret_cast<uintptr_t>(hidden) & 31u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+  if (w32)
+    k_permute<Vec32><<<(unsigned)grid, kPermuteThreads, 0, st>>>(a);
+  else
+    k_permute<uint4><<<(unsigned)grid, kPermuteThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

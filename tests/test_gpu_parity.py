@@ -209,13 +209,21 @@ def _hidden(w, seed=0):
     return torch.randn((w.N, w.hidden), generator=g, device="cuda", dtype=torch.float32).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("shared", [False, True])
-def test_dispatch_matches_oracle_small(shared):
-    w = get_config("tiny").replace(T=777, shared_expert=shared)
+@pytest.mark.parametrize("shared,hidden_dim,out_offset", [
+    (False, 256, 0), (True, 256, 0),   # 32-byte rows and buffers: 32-byte vectors
+    (False, 264, 0),                   # 528-byte rows: 16-byte vectors
+    (True, 256, 8),                    # output 16 bytes past a 32-byte boundary
+])
+def test_dispatch_matches_oracle_small(shared, hidden_dim, out_offset):
+    w = get_config("tiny").replace(T=777, shared_expert=shared, hidden=hidden_dim)
     ids = topk_ids(get_config("tiny"))[:, :777].copy()
     plan = gpu_plan(w, ids)
     hidden = _hidden(w)
-    out = plan.dispatch_layout(0, hidden)
+    rows = w.A + (w.N if shared else 0)
+    flat = torch.zeros(rows * w.hidden + out_offset, dtype=torch.bfloat16, device="cuda")
+    out = flat[out_offset:].view(rows, w.hidden)
+    assert (out.data_ptr() % 32 == 0) == (out_offset == 0)
+    plan.dispatch_layout(0, hidden, out=out)
     torch.cuda.synchronize()
     o = oracle_plan(w, ids)
     want = oracle.permute(o, hidden.view(torch.int16).cpu().numpy())

@@ -244,6 +244,35 @@ def test_invariants_full_configs(name):
     assert ratio <= 1.05 or p.cand_stop[0] == 1, (name, ratio, p.stop_name)
 
 
+def test_invariants_random_shapes():
+    # 150 small random problems across the supported shape space: ragged E/R,
+    # 0..8 slots, 1..16 experts per token (with and without repeats), every
+    # minimum quota, shared expert in both candidate modes
+    rng = np.random.default_rng(8080)
+    for case in range(150):
+        R = int(rng.integers(1, 13))
+        E = int(rng.integers(1, min(32 * R, 200) + 1))
+        K = int(rng.integers(1, min(E, 16) + 1))
+        T = int(rng.integers(0, 160))
+        S = int(rng.integers(0, 9))
+        m = int(rng.choice([1, 2, 5, 20]))
+        shared = bool(rng.integers(0, 2))
+        all_ranks = bool(rng.integers(0, 2))
+        p_e = rng.dirichlet(np.full(E, 0.3))
+        if rng.integers(0, 2):  # distinct experts per token
+            g = rng.gumbel(size=(R * T, E)) + np.log(p_e + 1e-12)
+            ids = np.argsort(-g, axis=1)[:, :K].reshape(R, T, K).astype(np.int32)
+        else:  # independent draws, repeats allowed
+            ids = rng.choice(E, size=(R, T, K), p=p_e).astype(np.int32)
+        p = oracle.plan(ids, E=E, S=S, m=m, J=16, shared_expert=shared, seed=case,
+                        bonus_permille=10, all_ranks=all_ranks)
+        check_plan(ids, E, S, m, Gmax=p.Gmax, G=p.G, W=p.W, inst_expert=p.inst_expert,
+                   inst_quota=p.inst_quota, inst_off=p.inst_off, dst_row=p.dst_row, cap=p.cap,
+                   stop=p.stop_name, shared_rank=p.shared_rank, shared_row=p.shared_row,
+                   all_ranks=all_ranks)
+        assert p.rows == R * T * K + (R * T if shared else 0)
+
+
 @pytest.mark.slow
 def test_invariants_stress():
     cfg = get_config("stress")

@@ -146,6 +146,31 @@ def test_plan_parity_random_shapes():
         compare_plan(g, o, w)
 
 
+def test_plan_parity_random_shapes_wide():
+    # the rest of the shape space: up to 8 slots and 16 experts per token,
+    # repeated experts in a token, Waterfill over all ranks
+    rng = np.random.default_rng(4242)
+    for case in range(30):
+        R = int(rng.integers(1, 40))
+        E = int(rng.integers(1, min(32 * R, 400) + 1))
+        K = int(rng.integers(1, min(E, 16) + 1))
+        T = int(rng.integers(0, 500))
+        S = int(rng.integers(4, 9))
+        m = int(rng.choice([1, 4, 32]))
+        shared = bool(rng.integers(0, 2))
+        all_ranks = bool(rng.integers(0, 2))
+        p_e = rng.dirichlet(np.full(E, 0.3))
+        if rng.integers(0, 2):
+            g = rng.gumbel(size=(R * T, E)) + np.log(p_e + 1e-12)
+            ids = np.argsort(-g, axis=1)[:, :K].reshape(R, T, K).astype(np.int32)
+        else:
+            ids = rng.choice(E, size=(R, T, K), p=p_e).astype(np.int32)
+        w = get_config("tiny").replace(R=R, E=E, K=K, T=T, S=S, m=m, J=16, shared_expert=shared,
+                                       waterfill_all_ranks=all_ranks)
+        o = oracle_plan(w, ids)
+        compare_plan(fetch(gpu_plan(w, ids)), o, w)
+
+
 def test_plan_parity_bad_ids_and_ragged_tail():
     w = get_config("tiny").replace(T=1000, shared_expert=True)
     ids = topk_ids(get_config("tiny"))[:, :1000].copy()

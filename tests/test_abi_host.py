@@ -7,7 +7,8 @@ import re
 
 import pytest
 
-from moe_expert_load_b200 import _abi, config_from_workload, ep_abi_version, ep_plan_workspace_bytes
+from moe_expert_load_b200 import (_abi, config_from_workload, ep_abi_version, ep_plan_workspace_bytes,
+                                  ep_status_string)
 from moe_expert_load_b200 import build as lib_build
 from moe_expert_load_b200 import EpError
 from workloads import CONFIGS, get_config
@@ -116,3 +117,44 @@ def test_product_never_touches_the_oracle():
     for path in glob.glob(os.path.join(pkg, "**", "*.*"), recursive=True):
         if path.endswith((".py", ".cu", ".cuh", ".h")):
             assert "oracle" not in open(path).read().lower(), path
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include <string.h>
+#include "ep_balance.h"
+int main(void) {
+  ep_config c;
+  memset(&c, 0, sizeof c);
+  c.num_ranks = 4; c.num_experts = 8; c.top_k = 2; c.tokens_per_rank = 1024;
+  c.slots_per_rank = 1; c.min_replica_quota = 64; c.hidden = 256; c.num_layers = 1;
+  c.num_cap_candidates = 16; c.expert_weight_elems = 3 * 256 * 512;
+  c.waterfill_bonus_permille = 10; c.waterfill_seed = 1;
+  size_t n = 0;
+  ep_status_t st = ep_plan_workspace_bytes(&c, &n);
+  c.num_ranks = 0;
+  size_t m = 0;
+  ep_status_t bad = ep_plan_workspace_bytes(&c, &m);
+  printf("%d %zu %d %s %d\n", (int)st, n, (int)bad, ep_status_string(bad), (int)ep_abi_version());
+  return 0;
+}
+"""
+
+
+def test_plain_c_caller_links_and_runs(tmp_path):
+    # the boundary is a C ABI: a C99 program includes the header, links the
+    # library and calls its host-only entry points (no GPU needed)
+    import subprocess
+
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(_abi.library_path())
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lep_b200", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    want = ep_plan_workspace_bytes(config_from_workload(get_config("tiny"), waterfill_seed=1))
+    assert out[0] == "0" and int(out[1]) == want
+    assert out[2] == "1" and " ".join(out[3:-1]) == ep_status_string(1)
+    assert int(out[-1]) == ep_abi_version()

@@ -150,10 +150,12 @@ struct CombineArgs {
   const float* w;        // [N][K]
   const int32_t* dst_row;
   const int32_t* shared_row;  // null without a shared expert
+  const int32_t* rank_base;   // [R+1]: rank_base[R] = rows of the layout
   void* out;             // [N][hidden] bf16 or fp32
   int64_t N;
   int row16;
   int K;
+  int R;
   int out_f32;
 };
 
@@ -179,14 +181,17 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(CombineArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int row16 = a.row16;
+  const int rows = a.rank_base[a.R];  // rows of the layout: anything else is not read
   for (int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < a.N; n += nw) {
     int d = -1;
     float wk = 0.f;
     if (lane < a.K) {
       d = a.dst_row[n * a.K + lane];
       wk = a.w[n * a.K + lane];
+      if (d >= rows) d = -1;
     }
-    const int ds = a.shared_row ? a.shared_row[n] : -1;
+    int ds = a.shared_row ? a.shared_row[n] : -1;
+    if (ds >= rows) ds = -1;
     for (int c0 = 0; c0 < row16; c0 += kCW * 32) {
       float acc[kCW * 8];
 #pragma unroll
@@ -489,6 +494,8 @@ cudaError_t launch_combine(const Dims& d, const LayerBuf& L, const void* x, cons
   a.w = w;
   a.dst_row = L.dst_row;
   a.shared_row = d.sh ? L.shared_row : nullptr;
+  a.rank_base = L.rank_base;
+  a.R = d.R;
   a.out = out;
   a.N = (int64_t)d.R * d.T;
   a.row16 = d.hidden * 2 / 16;

@@ -1156,19 +1156,22 @@ __global__ void __launch_bounds__(kFixThreads) k_fixup(Dims d, LayerBuf L, Scrat
     int4 v = row4[i];
     const uint32_t q = rk4[i];
     const int q0 = q & 0xffu, q1 = (q >> 8) & 0xffu, q2 = (q >> 16) & 0xffu, q3 = q >> 24;
-    if (q0 != kNoRank) v.x += s_rb[q0];
-    if (q1 != kNoRank) v.y += s_rb[q1];
-    if (q2 != kNoRank) v.z += s_rb[q2];
-    if (q3 != kNoRank) v.w += s_rb[q3];
+    // a rank byte is a rank below R, or kNoRank for a dropped assignment;
+    // anything else leaves the row alone
+    if (q0 < R) v.x += s_rb[q0];
+    if (q1 < R) v.y += s_rb[q1];
+    if (q2 < R) v.z += s_rb[q2];
+    if (q3 < R) v.w += s_rb[q3];
     row4[i] = v;
   }
   for (int64_t i = 4 * A4 + i0; i < A; i += stride) {
     const int q = s.asg_rank[i];
-    if (q != kNoRank) L.dst_row[i] += s_rb[q];
+    if (q < R) L.dst_row[i] += s_rb[q];
   }
   const int n = R * d.nsub;
   for (int64_t t = i0; t < N; t += stride) {
     const int c = L.shared_rank[t];
+    if ((unsigned)c >= (unsigned)R) continue;  // every pick is a rank; guard the tables anyway
     const int r = (int)t / d.T, tt = (int)t - r * d.T;
     L.shared_row[t] += s_sb[c] + s.wsub_cnt[(int64_t)c * n + r * d.nsub + tt / kPlanSubT];
   }

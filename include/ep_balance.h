@@ -291,9 +291,14 @@ EP_API ep_status_t ep_waterfill(int32_t R, int32_t T, int32_t K, const int32_t* 
  * (4 MiB) that every GPU loading the library holds until the process exits;
  * larger shapes return EP_ERR_UNSUPPORTED.  The first call on each device looks
  * up the array's address (cudaGetSymbolAddress) — make that first call before
- * any stream capture.  All calls on a device share the array; calls that
- * overlap on the GPU race and must be serialised by the caller.  Limits: R >= 1,
- * 1 <= E <= 1024, 1 <= K <= 16, T >= 0, R*T*K < 2^31.  Asynchronous on `stream`.
+ * any stream capture.  The address is cached with the id of the CUDA context
+ * it belongs to; after a device reset the next call looks it up again, so make
+ * that call, too, before any capture.  All calls on a device share the array;
+ * calls that overlap on the GPU race and must be serialised by the caller.
+ * Limits: R >= 1, 1 <= E <= 1024, 1 <= K <= 16, T >= 0, R*T*K < 2^31,
+ * R*E < 2^31.  Asynchronous on `stream`; EP_ERR_CUDA reports a failure of this
+ * call's own memset or launches only (an error left pending by earlier,
+ * unrelated work is not reported and not cleared).
  */
 #define EP_LOAD_STATIC_MAX_SCRATCH (1 << 20)
 EP_API ep_status_t ep_load_matrix_static(int32_t R, int32_t E, int32_t K, int32_t T,

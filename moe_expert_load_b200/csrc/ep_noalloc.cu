@@ -14,6 +14,13 @@
 // last call's contents; each call overwrites every entry it later reads, so
 // nothing in it has to start at zero.  Calls whose executions overlap on the
 // GPU (two streams, or two host threads) race on the array: serialise them.
+//
+// Host code cannot use the array's name as a device address, so the address is
+// looked up with cudaGetSymbolAddress once per device and cached together with
+// the unique id of the CUDA context it belongs to.  After a device reset the
+// module is loaded again in a new context, possibly at another address; the
+// next call sees the new context id and looks the address up again.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -31,23 +38,60 @@ constexpr unsigned kFull = 0xffffffffu;
 static __device__ __align__(256) int32_t g_load_scratch[EP_LOAD_STATIC_MAX_SCRATCH];
 
 std::mutex g_setup_mu;
-int32_t* g_scratch_addr[kMaxDevices] = {};
+
+struct CachedAddress {
+  int32_t* addr = nullptr;
+  unsigned long long ctx_id = 0;  // unique id of the context the address belongs to
+};
+CachedAddress g_scratch_addr[kMaxDevices];
+
+// Driver entry points, fetched through the runtime (no link against libcuda).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+bool g_driver_fns_tried = false;
+
+// Unique id of the current context (0 if it cannot be read; ids are never 0).
+unsigned long long current_context_id() {
+  if (!g_driver_fns_tried) {
+    g_driver_fns_tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f);
+  }
+  if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of g_load_scratch on the current device, looked up once per
-// device (host code may not use the array's name as an address).
+// device and context (host code may not use the array's name as an address).
 cudaError_t scratch_address(int32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_addr[dev]) {
+  CachedAddress& c = g_scratch_addr[dev];
+  const unsigned long long id = c.addr ? current_context_id() : 0;
+  if (!c.addr || id == 0 || id != c.ctx_id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_load_scratch);
+    e = cudaGetSymbolAddress(&p, g_load_scratch);  // makes the device's context current
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = static_cast<int32_t*>(p);
+    c.addr = static_cast<int32_t*>(p);
+    c.ctx_id = current_context_id();
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return cudaSuccess;
 }
 
@@ -101,7 +145,8 @@ extern "C" ep_status_t ep_load_matrix_static(int32_t R, int32_t E, int32_t K, in
                                              const int32_t* d_topk_ids, int32_t* d_load,
                                              int32_t* d_status, void* stream) {
   if (R < 1 || E < 1 || K < 1 || T < 0) return EP_ERR_INVALID_ARGUMENT;
-  if (E > ep::kMaxE || K > ep::kMaxK || (int64_t)R * T * K >= (int64_t)INT32_MAX)
+  if (E > ep::kMaxE || K > ep::kMaxK || (int64_t)R * T * K >= (int64_t)INT32_MAX ||
+      (int64_t)R * E >= (int64_t)INT32_MAX)
     return EP_ERR_UNSUPPORTED;
   const int nsub = (T + ep::kSubT - 1) / ep::kSubT;
   if ((int64_t)R * nsub * E > (int64_t)EP_LOAD_STATIC_MAX_SCRATCH) return EP_ERR_UNSUPPORTED;
@@ -111,10 +156,21 @@ extern "C" ep_status_t ep_load_matrix_static(int32_t R, int32_t E, int32_t K, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d_status && cudaMemsetAsync(d_status, 0, sizeof(int32_t), st) != cudaSuccess)
     return EP_ERR_CUDA;
+  // each launch's own return code: an error left pending by unrelated earlier
+  // work is neither reported here nor cleared
   const int nwarps = R * nsub;
-  if (nwarps > 0)
-    k_hist_static<<<(nwarps + kWarps - 1) / kWarps, kWarps * 32, sizeof(int32_t) * kWarps * E, st>>>(
-        d_topk_ids, R, E, K, T, nsub, scratch, d_status);
-  k_load_static<<<(R * E + 255) / 256, 256, 0, st>>>(R, E, nsub, scratch, d_load);
-  return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+  if (nwarps > 0) {
+    void* args[] = {&d_topk_ids, &R, &E, &K, &T, const_cast<int*>(&nsub), &scratch, &d_status};
+    if (cudaLaunchKernel(reinterpret_cast<const void*>(k_hist_static),
+                         dim3((unsigned)((nwarps + kWarps - 1) / kWarps)), dim3(kWarps * 32), args,
+                         sizeof(int32_t) * kWarps * E, st) != cudaSuccess)
+      return EP_ERR_CUDA;
+  }
+  const int32_t* cscratch = scratch;
+  void* args2[] = {&R, &E, const_cast<int*>(&nsub), &cscratch, &d_load};
+  if (cudaLaunchKernel(reinterpret_cast<const void*>(k_load_static),
+                       dim3((unsigned)(((int64_t)R * E + 255) / 256)), dim3(256), args2, 0, st) !=
+      cudaSuccess)
+    return EP_ERR_CUDA;
+  return EP_OK;
 }

@@ -73,6 +73,26 @@ def test_static_load_matrix_matches_balance_layer_twice():
     np.testing.assert_array_equal(results[0][0].cpu().numpy(), ref)
 
 
+@pytest.mark.gpu
+def test_static_load_matrix_ragged_tail_and_empty():
+    # T = 1000 leaves a partial last sub-chunk of 104 tokens and K = 3 makes
+    # the ids of a sub-chunk end inside a 32-lane pass; T = 0 writes zeros
+    rng = np.random.default_rng(17)
+    R, E, K, T = 3, 40, 3, 1000
+    ids_np = rng.integers(0, E, size=(R, T, K)).astype(np.int32)
+    ids_np[2, 999, 2] = E + 1  # the very last id is out of range
+    for _ in range(2):  # twice in a row on the shared array
+        load, status = _static_load(torch.from_numpy(ids_np).cuda(), E)
+        torch.cuda.synchronize()
+        ref = np.stack([np.bincount(r.ravel()[r.ravel() < E], minlength=E) for r in ids_np])
+        np.testing.assert_array_equal(load.cpu().numpy(), ref)
+        assert int(status.item()) == 1
+    empty = torch.empty((5, 0, 4), dtype=torch.int32, device="cuda")
+    load, status = _static_load(empty, 16)
+    torch.cuda.synchronize()
+    assert not load.any() and int(status.item()) == 0
+
+
 def test_static_load_matrix_rejects_shapes_beyond_its_scratch():
     f = _fn()
     w = get_config("stress")  # 72 * 128 * 256 sub-chunk counts > 2^20
@@ -80,3 +100,5 @@ def test_static_load_matrix_rejects_shapes_beyond_its_scratch():
     assert f(w.R, w.E, w.K, w.T, None, None, None, None) == 2
     assert f(0, 8, 2, 10, None, None, None, None) == 1
     assert f(4, 8, 2, 10, None, None, None, None) == 1  # null pointers
+    # with T = 0 the scratch bound holds for any R, so R * E itself is bounded
+    assert f(3_000_000, 1024, 2, 0, None, None, None, None) == 2

@@ -34,6 +34,8 @@ class _Cfg(ctypes.Structure):
         ("S", ctypes.c_int32), ("m", ctypes.c_int32), ("J", ctypes.c_int32),
         ("shared_expert", ctypes.c_int32), ("bonus_permille", ctypes.c_int32),
         ("all_ranks", ctypes.c_int32), ("seed", ctypes.c_uint64),
+        ("sampling", ctypes.c_int32), ("iter_limit", ctypes.c_int32),
+        ("sampling_seed", ctypes.c_uint64),
     ]
 
 
@@ -43,6 +45,7 @@ class _Stats(ctypes.Structure):
         ("stop_reason", ctypes.c_int32), ("cap", ctypes.c_int64), ("A", ctypes.c_int64),
         ("before_max", ctypes.c_int64), ("after_max", ctypes.c_int64),
         ("replicas", ctypes.c_int32), ("status", ctypes.c_int32), ("rows", ctypes.c_int64),
+        ("realized_max", ctypes.c_int64),
     ]
 
 
@@ -54,7 +57,7 @@ def _load():
     if _lib is None:
         lib = ctypes.CDLL(_build.build())
         P = ctypes.c_void_p
-        lib.orc_plan.argtypes = [ctypes.POINTER(_Cfg), P] + [P] * 14 + [ctypes.POINTER(_Stats)]
+        lib.orc_plan.argtypes = [ctypes.POINTER(_Cfg), P] + [P] * 15 + [ctypes.POINTER(_Stats)]
         lib.orc_plan.restype = ctypes.c_int
         lib.orc_load_matrix.argtypes = [ctypes.c_int32] * 4 + [P, P]
         lib.orc_load_matrix.restype = ctypes.c_int64
@@ -99,7 +102,8 @@ class Plan:
     W0: np.ndarray  # [R]
     W: np.ndarray  # [R]
     inst_expert: np.ndarray  # [R][G] int32
-    inst_quota: np.ndarray  # [R][G] int64
+    inst_quota: np.ndarray  # [R][G] int64: the solve's split (shared column: its rows)
+    inst_count: np.ndarray  # [R][G] int64: rows each instance receives
     inst_off: np.ndarray  # [R*G+1] int64
     dst_inst: np.ndarray  # [R][T][K] int32
     dst_row: np.ndarray  # [R][T][K] int64
@@ -117,6 +121,7 @@ class Plan:
     replicas: int
     status: int
     rows: int
+    realized_max: int
 
     @property
     def stop_name(self) -> str:
@@ -128,14 +133,20 @@ def gmax(E: int, R: int) -> int:
 
 
 def plan(ids: np.ndarray, *, E: int, S: int, m: int, J: int = 16, shared_expert: bool = False,
-         seed: int = 0, bonus_permille: int = 10, all_ranks: bool = False) -> Plan:
-    """Whole balance + dispatch plan of one layer from gate ids [R][T][K]."""
+         seed: int = 0, bonus_permille: int = 10, all_ranks: bool = False, sampling: bool = False,
+         sampling_seed: int = 0, iter_limit: int = 0) -> Plan:
+    """Whole balance + dispatch plan of one layer from gate ids [R][T][K].
+
+    sampling: each (token, k) draws an instance of its expert with probability
+    quota / expert total (the LPLB-style dispatch) instead of the local-first
+    rerouting; iter_limit > 0 replaces the greedy's iteration bound."""
     lib = _load()
     ids = np.ascontiguousarray(ids, dtype=np.int32)
     R, T, K = ids.shape
     cfg = _Cfg(R=R, E=E, K=K, T=T, S=S, m=m, J=J, shared_expert=int(bool(shared_expert)),
                bonus_permille=bonus_permille, all_ranks=int(bool(all_ranks)),
-               seed=seed & 0xFFFFFFFFFFFFFFFF)
+               seed=seed & 0xFFFFFFFFFFFFFFFF, sampling=int(bool(sampling)),
+               iter_limit=int(iter_limit), sampling_seed=sampling_seed & 0xFFFFFFFFFFFFFFFF)
     Gm = gmax(E, R)
     G = Gm + S + (1 if shared_expert else 0)
     L = np.zeros((R, E), np.int64)
@@ -144,6 +155,7 @@ def plan(ids: np.ndarray, *, E: int, S: int, m: int, J: int = 16, shared_expert:
     W = np.zeros(R, np.int64)
     inst_expert = np.zeros((R, G), np.int32)
     inst_quota = np.zeros((R, G), np.int64)
+    inst_count = np.zeros((R, G), np.int64)
     inst_off = np.zeros(R * G + 1, np.int64)
     dst_inst = np.zeros((R, T, K), np.int32)
     dst_row = np.zeros((R, T, K), np.int64)
@@ -154,17 +166,19 @@ def plan(ids: np.ndarray, *, E: int, S: int, m: int, J: int = 16, shared_expert:
     cand_stop = np.zeros(J, np.int32)
     st = _Stats()
     rc = lib.orc_plan(ctypes.byref(cfg), _p(ids), _p(L), _p(Tot), _p(W0), _p(W), _p(inst_expert),
-                      _p(inst_quota), _p(inst_off), _p(dst_inst), _p(dst_row), _p(shared_rank),
+                      _p(inst_quota), _p(inst_count), _p(inst_off), _p(dst_inst), _p(dst_row),
+                      _p(shared_rank),
                       _p(shared_row), _p(cand_maxW), _p(cand_repl), _p(cand_stop), ctypes.byref(st))
     if rc != 0:
         raise ValueError(f"oracle rejected the configuration (code {rc})")
     return Plan(R=R, E=E, K=K, T=T, S=S, Gmax=st.Gmax, G=st.G, L=L, Tot=Tot, W0=W0, W=W,
-                inst_expert=inst_expert, inst_quota=inst_quota, inst_off=inst_off,
+                inst_expert=inst_expert, inst_quota=inst_quota, inst_count=inst_count,
+                inst_off=inst_off,
                 dst_inst=dst_inst, dst_row=dst_row, shared_rank=shared_rank, shared_row=shared_row,
                 cand_maxW=cand_maxW, cand_repl=cand_repl, cand_stop=cand_stop,
                 cap_idx=st.cap_idx, cap=st.cap, stop_reason=st.stop_reason, A=st.A,
                 before_max=st.before_max, after_max=st.after_max, replicas=st.replicas,
-                status=st.status, rows=st.rows)
+                status=st.status, rows=st.rows, realized_max=st.realized_max)
 
 
 def load_matrix(ids: np.ndarray, E: int):

@@ -22,6 +22,10 @@
  *     - section "Reusing the forward plan": backward re-stages replica weights
  *       from the cached plan, reduces replica gradients into the native
  *       expert's gradient buffer and then clears the replica buffer.
+ *   "Waterfill and LPLB" page, section "LPLB": the per-expert split over
+ *     its physical instances, normalised to a probability distribution, from
+ *     which every token routed to a replicated expert samples one instance
+ *     (the sampling rerouting mode, in place of local-first rerouting);
  *   "Waterfill and LPLB" page, section "Waterfill": the waterline
  *     H = ceil((sum_r L_r + N) / R), slack S_r = max(H - L_r, 0), per-token
  *     sampling proportional to slack among the local rank and the ranks the
@@ -62,6 +66,10 @@ typedef struct {
   int32_t bonus_permille; /* local preference of the Waterfill draw */
   int32_t all_ranks;      /* 1: Waterfill candidates are all ranks, not only visited ones */
   uint64_t seed;          /* Waterfill draw seed */
+  int32_t sampling;       /* 1: every (token, k) samples an instance of its expert with
+                             probability proportional to the instance's quota */
+  int32_t iter_limit;     /* > 0: replaces the greedy's iteration bound (tests of the bound) */
+  uint64_t sampling_seed; /* seed of the per-assignment draw of the sampling mode */
 } orc_cfg;
 
 typedef struct {
@@ -75,6 +83,7 @@ typedef struct {
   int32_t replicas;       /* replicas created */
   int32_t status;         /* ST_* bits */
   int64_t rows;           /* total dispatch rows (A, plus N with a shared expert) */
+  int64_t realized_max;   /* max per-rank routed rows actually dispatched */
 } orc_stats;
 
 /* ---- O1: native placement, contiguous balanced blocks ------------------ */
@@ -211,7 +220,7 @@ static void greedy(const orc_cfg* c, const int64_t* Tot, const int64_t* W0, int6
   for (int64_t i = 0; i < (int64_t)R * S; ++i) { g->slot_e[i] = -1; g->slot_q[i] = 0; }
   g->replicas = 0;
   g->stop = -1;
-  const int64_t iter_cap = 4 * ((int64_t)R * S + R + E) + 64;
+  const int64_t iter_cap = c->iter_limit > 0 ? c->iter_limit : 4 * ((int64_t)R * S + R + E) + 64;
   for (int64_t it = 0;; ++it) {
     if (it >= iter_cap) { g->stop = STOP_ITER_CAP; break; }
     /* 1. most loaded rank that is not stuck, smallest index on ties */
@@ -295,8 +304,10 @@ static void greedy(const orc_cfg* c, const int64_t* Tot, const int64_t* W0, int6
  *   Tot      [E]               per-expert totals
  *   W0, W    [R]               per-rank load before / after the solve (O3, O4)
  *   inst_expert [R][G] int32   instance table (O5); -1 empty, E = shared column
- *   inst_quota  [R][G]         quota of each instance
- *   inst_off    [R*G+1]        exclusive prefix of quotas, in instance order (O8)
+ *   inst_quota  [R][G]         quota of each instance (the solve's split)
+ *   inst_count  [R][G]         rows each instance receives: its quota, except in the
+ *                              sampling mode, where it is the number of draws it got
+ *   inst_off    [R*G+1]        exclusive prefix of inst_count, in instance order (O8)
  *   dst_inst    [R][T][K]      global instance index of each assignment, -1 if invalid
  *   dst_row     [R][T][K]      dispatch row of each assignment (O7, O8), -1 if invalid
  *   shared_rank [R][T]         Waterfill rank of each token's shared slot (O10), or NULL
@@ -304,9 +315,10 @@ static void greedy(const orc_cfg* c, const int64_t* Tot, const int64_t* W0, int6
  *   cand_maxW, cand_repl, cand_stop [J]   each cap candidate's result
  */
 int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int64_t* W0,
-             int64_t* W, int32_t* inst_expert, int64_t* inst_quota, int64_t* inst_off,
-             int32_t* dst_inst, int64_t* dst_row, int32_t* shared_rank, int64_t* shared_row,
-             int64_t* cand_maxW, int32_t* cand_repl, int32_t* cand_stop, orc_stats* st) {
+             int64_t* W, int32_t* inst_expert, int64_t* inst_quota, int64_t* inst_count,
+             int64_t* inst_off, int32_t* dst_inst, int64_t* dst_row, int32_t* shared_rank,
+             int64_t* shared_row, int64_t* cand_maxW, int32_t* cand_repl, int32_t* cand_stop,
+             orc_stats* st) {
   const int32_t R = c->R, E = c->E, K = c->K, T = c->T, S = c->S;
   if (R < 1 || E < 1 || K < 1 || T < 0 || S < 0 || c->m < 1 || c->J < 1) return ORC_BAD_ARG;
   const int32_t Gmax = orc_gmax(E, R);
@@ -464,20 +476,72 @@ int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int
   int64_t* cur_seg = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
   int64_t* cur_used = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
   int64_t* dst_pos = (int64_t*)malloc(sizeof(int64_t) * ((size_t)R * T * K + 1));
-  for (int32_t r = 0; r < R; ++r) {
-    for (int32_t e = 0; e < E; ++e) { cur_seg[e] = tmp_ptr[(int64_t)r * E + e]; cur_used[e] = 0; }
-    for (int64_t a = 0; a < (int64_t)T * K; ++a) {
-      const int64_t idx = (int64_t)r * T * K + a;
-      const int32_t e = ids[idx];
-      if (e < 0 || e >= E) { dst_inst[idx] = -1; dst_pos[idx] = -1; continue; }
-      while (cur_used[e] == seg_cnt[cur_seg[e]]) { ++cur_seg[e]; cur_used[e] = 0; }
-      dst_inst[idx] = seg_inst[cur_seg[e]];
-      dst_pos[idx] = seg_pos[cur_seg[e]] + cur_used[e];
-      ++cur_used[e];
+  if (!c->sampling) {
+    for (int32_t r = 0; r < R; ++r) {
+      for (int32_t e = 0; e < E; ++e) { cur_seg[e] = tmp_ptr[(int64_t)r * E + e]; cur_used[e] = 0; }
+      for (int64_t a = 0; a < (int64_t)T * K; ++a) {
+        const int64_t idx = (int64_t)r * T * K + a;
+        const int32_t e = ids[idx];
+        if (e < 0 || e >= E) { dst_inst[idx] = -1; dst_pos[idx] = -1; continue; }
+        while (cur_used[e] == seg_cnt[cur_seg[e]]) { ++cur_seg[e]; cur_used[e] = 0; }
+        dst_inst[idx] = seg_inst[cur_seg[e]];
+        dst_pos[idx] = seg_pos[cur_seg[e]] + cur_used[e];
+        ++cur_used[e];
+      }
     }
   }
 
-  /* O10: Waterfill shared-expert slot of each token */
+  /* Sampling mode ("Waterfill and LPLB" page, section "LPLB"): the solve's
+   * split of each expert over its instances, divided by the expert's total, is
+   * a probability distribution over the instances; every (token, k) draws one
+   * instance from it independently, and an expert with a single instance maps
+   * to it without a draw.  The draw is made reproducible with a counter-based
+   * hash of the assignment index a = (r*T + t)*K + k:
+   * h = SplitMix64(sampling_seed + a), u = ((h >> 32) * total) >> 32, and the
+   * pick is the first instance, in instance order, whose running quota sum
+   * exceeds u.  Rows of an instance keep the order (source rank, t, k). */
+  int64_t* run = (int64_t*)calloc((size_t)R * G, sizeof(int64_t));
+  if (c->sampling) {
+    /* instances of each expert in instance order (natives and replicas) */
+    int64_t* eptr = (int64_t*)calloc((size_t)E + 1, sizeof(int64_t));
+    int32_t* elist = (int32_t*)malloc(sizeof(int32_t) * ((size_t)R * G + 1));
+    for (int64_t i = 0; i < (int64_t)R * G; ++i) {
+      const int32_t e = inst_expert[i];
+      if (e >= 0 && e < E) eptr[e + 1] += 1;
+    }
+    for (int32_t e = 0; e < E; ++e) eptr[e + 1] += eptr[e];
+    int64_t* fill = (int64_t*)malloc(sizeof(int64_t) * ((size_t)E + 1));
+    for (int32_t e = 0; e <= E; ++e) fill[e] = eptr[e];
+    for (int64_t i = 0; i < (int64_t)R * G; ++i) {
+      const int32_t e = inst_expert[i];
+      if (e >= 0 && e < E) elist[fill[e]++] = (int32_t)i;
+    }
+    for (int64_t idx = 0; idx < (int64_t)R * T * K; ++idx) {
+      const int32_t e = ids[idx];
+      if (e < 0 || e >= E) { dst_inst[idx] = -1; dst_pos[idx] = -1; continue; }
+      const int64_t n = eptr[e + 1] - eptr[e];
+      int32_t pick = elist[eptr[e]];
+      if (n > 1) {
+        const uint64_t h = orc_splitmix64(c->sampling_seed + (uint64_t)idx);
+        const uint64_t u = ((h >> 32) * (uint64_t)Tot[e]) >> 32;
+        int64_t acc = 0;
+        for (int64_t j = 0; j < n; ++j) {
+          acc += inst_quota[elist[eptr[e] + j]];
+          if ((uint64_t)acc > u) { pick = elist[eptr[e] + j]; break; }
+        }
+      }
+      dst_inst[idx] = pick;
+      dst_pos[idx] = run[pick]++; /* assignments are visited in (r, t, k) order */
+    }
+    free(eptr);
+    free(elist);
+    free(fill);
+  }
+
+  /* O10: Waterfill shared-expert slot of each token.  The load score of a
+   * rank is its routed load W after the solve; in the sampling mode that is
+   * the planned (expected) load, the realised one being known only after every
+   * draw. */
   int64_t* shared_cnt = (int64_t*)calloc((size_t)R, sizeof(int64_t));
   if (sh) {
     int64_t H, B;
@@ -502,9 +566,21 @@ int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int
     for (int32_t q = 0; q < R; ++q) inst_quota[(int64_t)q * G + Gmax + S] = shared_cnt[q];
   }
 
+  /* rows each instance receives: the quota, or the draws it got */
+  for (int64_t i = 0; i < (int64_t)R * G; ++i) {
+    const int shared_col = sh && (i % G) == Gmax + S;
+    inst_count[i] = (c->sampling && !shared_col) ? run[i] : inst_quota[i];
+  }
+  st->realized_max = 0;
+  for (int32_t q = 0; q < R; ++q) {
+    int64_t w = 0;
+    for (int32_t col = 0; col < Gmax + S; ++col) w += inst_count[(int64_t)q * G + col];
+    if (w > st->realized_max) st->realized_max = w;
+  }
+
   /* O8: row layout */
   inst_off[0] = 0;
-  for (int64_t i = 0; i < (int64_t)R * G; ++i) inst_off[i + 1] = inst_off[i] + inst_quota[i];
+  for (int64_t i = 0; i < (int64_t)R * G; ++i) inst_off[i + 1] = inst_off[i] + inst_count[i];
   st->rows = inst_off[(int64_t)R * G];
   for (int64_t a = 0; a < (int64_t)R * T * K; ++a)
     dst_row[a] = dst_inst[a] < 0 ? -1 : inst_off[dst_inst[a]] + dst_pos[a];
@@ -519,6 +595,7 @@ int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int
   }
 
   free(shared_cnt);
+  free(run);
   free(dst_pos);
   free(cur_seg);
   free(cur_used);

@@ -158,3 +158,62 @@ def check_plan(ids: np.ndarray, E: int, S: int, m: int, *, Gmax: int, G: int, W,
                 assert rr[0] == inst_off[q * G + Gmax + S]
     return dict(L=L, Tot=Tot)
 
+
+
+def check_sampled_rows(ids: np.ndarray, E: int, *, Gmax: int, G: int, S: int, inst_expert,
+                       inst_quota, inst_count, inst_off, dst_row, shared_rank=None,
+                       shared_row=None):
+    """Rows of the sampling rerouting mode ("Waterfill and LPLB" page, section
+    "LPLB": each token of a replicated expert samples one of its physical
+    instances).  Whatever the draws, the rows must be a bijection, each row
+    must sit in an instance of its token's expert, the rows an instance
+    receives must be what the layout gives it, an instance the split gives no
+    tokens can never be drawn, an expert with one instance keeps all its
+    tokens there, and rows inside an instance follow (source rank, t, k)."""
+    ids = np.asarray(ids)
+    R, T, K = ids.shape
+    inst_expert = np.asarray(inst_expert).reshape(R, G)
+    inst_quota = np.asarray(inst_quota, dtype=np.int64).reshape(R, G)
+    inst_count = np.asarray(inst_count, dtype=np.int64).reshape(R, G)
+    inst_off = np.asarray(inst_off, dtype=np.int64).reshape(-1)
+    dst_row = np.asarray(dst_row, dtype=np.int64).reshape(R, T, K)
+    sh = G - Gmax - S
+    valid = (ids >= 0) & (ids < E)
+    Tot = np.bincount(ids[valid].ravel(), minlength=E)
+    assert inst_off[0] == 0 and (np.diff(inst_off) == inst_count.reshape(-1)).all()
+    rows = int(inst_off[-1])
+    d = dst_row[valid]
+    assert (dst_row[~valid] == -1).all()
+    all_rows = d if not sh else np.concatenate([d, np.asarray(shared_row, np.int64).ravel()])
+    assert len(all_rows) == rows
+    assert (np.sort(all_rows) == np.arange(rows)).all(), "rows are a bijection"
+    inst_of_row = np.searchsorted(inst_off, np.arange(rows), side="right") - 1
+    flat_e = inst_expert.reshape(-1)
+    inst_a = inst_of_row[d]
+    assert (flat_e[inst_a] == ids[valid]).all(), "row hosts another expert"
+    n_inst = np.zeros(E, np.int64)
+    got = np.zeros(E, np.int64)
+    for q in range(R):
+        for col in range(Gmax + S):
+            e = inst_expert[q, col]
+            if e >= 0:
+                n_inst[e] += 1
+                got[e] += inst_count[q, col]
+                if inst_quota[q, col] == 0:
+                    assert inst_count[q, col] == 0, "an instance with no quota was drawn"
+    assert (got == Tot).all(), "every assignment of an expert lands in one of its instances"
+    for q in range(R):
+        for col in range(Gmax + S):
+            e = inst_expert[q, col]
+            if e >= 0 and n_inst[e] == 1:
+                assert inst_count[q, col] == Tot[e], "single instance keeps all its tokens"
+    flat_idx = np.arange(R * T * K).reshape(R, T, K)[valid]
+    order = np.argsort(d)
+    same = inst_a[order][1:] == inst_a[order][:-1]
+    src = flat_idx[order]
+    assert (src[1:][same] > src[:-1][same]).all(), "row order inside an instance"
+    if sh:
+        sr = np.asarray(shared_rank).reshape(R, T)
+        counts = np.bincount(sr.ravel(), minlength=R)
+        assert (inst_count[:, Gmax + S] == counts).all()
+        assert (inst_quota[:, Gmax + S] == counts).all()

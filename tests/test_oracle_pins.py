@@ -619,3 +619,133 @@ def test_greedy_split_is_never_below_the_lp_bound(name):
     M, _ = min_max_split(p.Tot, p.inst_expert, p.Gmax, p.S, m_replica=cfg.m)
     assert p.after_max >= M - 1e-6
     assert p.after_max <= 1.06 * M  # and close to it on these workloads
+
+
+# ---- sampling rerouting mode ("Waterfill and LPLB" page, section "LPLB") --------
+def _fig_ep4():
+    case = next(c for c in _golden("quota_worked_examples.json")["cases"] if c["name"] == "fig_ep4")
+    return case, np.array(case["ids"], dtype=np.int32).reshape(case["R"], case["T"], case["K"])
+
+
+def test_sampling_hand_worked_draws():
+    g = _golden("sampling_worked_example.json")
+    case, ids = _fig_ep4()
+    for d in g["draws"]:
+        p = oracle.plan(ids, E=case["E"], S=case["S"], m=case["m"], J=case["J"], sampling=True,
+                        sampling_seed=int(d["seed"]))
+        assert p.dst_inst[d["r"], d["t"], d["k"]] == d["instance"], d
+
+
+def _sampled(cfg, ids, seed=77, **kw):
+    return _plan_cfg(cfg, ids, sampling=True, sampling_seed=seed, **kw)
+
+
+def _check_sampled(p, ids, E, S):
+    from tests.invariants import check_sampled_rows
+
+    check_sampled_rows(ids, E, Gmax=p.Gmax, G=p.G, S=S, inst_expert=p.inst_expert,
+                       inst_quota=p.inst_quota, inst_count=p.inst_count, inst_off=p.inst_off,
+                       dst_row=p.dst_row, shared_rank=p.shared_rank, shared_row=p.shared_row)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen", "dsv3"])
+def test_sampling_keeps_the_solve_and_gives_valid_rows(name):
+    cfg = get_config(name)
+    ids = topk_ids(cfg)
+    det = _plan_cfg(cfg, ids)
+    p = _sampled(cfg, ids)
+    # the solve is the same in both modes; only the token-to-instance step differs
+    for f in ("L", "Tot", "W0", "W", "inst_expert", "cand_maxW", "cand_repl", "cand_stop"):
+        np.testing.assert_array_equal(getattr(p, f), getattr(det, f), err_msg=f)
+    sc = det.Gmax + det.S  # the shared column's quota depends on the routed ranks
+    np.testing.assert_array_equal(p.inst_quota[:, :sc], det.inst_quota[:, :sc])
+    assert (p.cap_idx, p.replicas, p.after_max, p.A) == (det.cap_idx, det.replicas, det.after_max, det.A)
+    _check_sampled(p, ids, cfg.E, cfg.S)
+    np.testing.assert_array_equal(det.inst_count, det.inst_quota)
+    assert det.realized_max == det.after_max
+    routed = p.inst_count[:, :sc].sum(axis=1)
+    assert p.realized_max == routed.max()
+    if p.replicas:  # the draws do move tokens off the deterministic rows
+        assert (p.dst_inst != det.dst_inst).any()
+
+
+def test_sampling_without_slots_is_the_counting_sort():
+    # one instance per expert: no draw, rows in (expert, source, t, k) order
+    rng = np.random.default_rng(12)
+    for _ in range(10):
+        R = int(rng.integers(1, 6))
+        E = int(rng.integers(1, 16))
+        ids = rng.integers(0, E, size=(R, int(rng.integers(0, 40)), int(rng.integers(1, 4)))).astype(np.int32)
+        p = oracle.plan(ids, E=E, S=0, m=2, J=4, sampling=True, sampling_seed=5)
+        expect = np.empty(ids.size, np.int64)
+        expect[np.argsort(ids.ravel(), kind="stable")] = np.arange(ids.size)
+        assert (p.dst_row.ravel() == expect).all()
+
+
+def test_sampling_proportional_to_quota():
+    # each replicated expert's tokens split over its instances in proportion
+    # to the quotas: every realised count within 5 binomial sigma of its quota
+    cfg = get_config("qwen")
+    ids = topk_ids(cfg)
+    p = _sampled(cfg, ids, seed=2026)
+    checked = 0
+    for e in range(cfg.E):
+        cols = np.argwhere(p.inst_expert[:, :p.Gmax + cfg.S] == e)
+        if len(cols) < 2:
+            continue
+        tot = int(p.Tot[e])
+        for q, c in cols:
+            pr = p.inst_quota[q, c] / tot
+            sigma = np.sqrt(tot * pr * (1 - pr))
+            assert abs(int(p.inst_count[q, c]) - int(p.inst_quota[q, c])) <= 5 * sigma + 1
+            checked += 1
+    assert checked > p.replicas  # every replica plus its native
+
+
+def test_sampling_draw_depends_only_on_seed_and_assignment():
+    cfg = get_config("tiny")
+    ids = topk_ids(cfg)
+    a = _sampled(cfg, ids, seed=3)
+    b = _sampled(cfg, ids, seed=3)
+    c = _sampled(cfg, ids, seed=4)
+    np.testing.assert_array_equal(a.dst_row, b.dst_row)
+    assert (a.dst_inst != c.dst_inst).any()
+    # swap two tokens of one rank: loads, quotas and every other draw stay
+    ids2 = ids.copy()
+    ids2[1, [10, 700]] = ids2[1, [700, 10]]
+    d = _sampled(cfg, ids2, seed=3)
+    np.testing.assert_array_equal(d.inst_quota, a.inst_quota)
+    keep = np.ones(ids.shape, bool)
+    keep[1, [10, 700]] = False
+    np.testing.assert_array_equal(d.dst_inst[keep], a.dst_inst[keep])
+
+
+def test_sampling_random_shapes():
+    rng = np.random.default_rng(31)
+    for _ in range(40):
+        R = int(rng.integers(1, 9))
+        E = int(rng.integers(1, min(32 * R, 60) + 1))
+        K = int(rng.integers(1, 6))
+        T = int(rng.integers(0, 120))
+        S = int(rng.integers(0, 4))
+        shared = bool(rng.integers(0, 2))
+        ids = rng.choice(E, size=(R, T, K), p=rng.dirichlet(np.full(E, 0.3))).astype(np.int32)
+        if T and rng.integers(0, 2):
+            ids[0, 0, 0] = E  # a dropped id
+        p = oracle.plan(ids, E=E, S=S, m=int(rng.choice([1, 4])), J=8, shared_expert=shared,
+                        sampling=True, sampling_seed=int(rng.integers(0, 2**63)))
+        _check_sampled(p, ids, E, S)
+
+
+# ---- the greedy's iteration bound ----------------------------------------------
+def test_iteration_limit_stops_the_greedy_and_keeps_a_valid_plan():
+    cfg = get_config("qwen")
+    ids = topk_ids(cfg)
+    full = _plan_cfg(cfg, ids)
+    assert full.replicas >= 3
+    p = _plan_cfg(cfg, ids, iter_limit=2)
+    assert p.status & oracle.ST_ITER_CAP
+    assert (p.cand_stop == 3).all()  # every candidate needed more than two moves
+    assert (p.cand_repl <= 2).all()
+    assert p.stop_name == "ITER_CAP"
+    _check(p, ids, cfg.E, cfg.S, cfg.m)

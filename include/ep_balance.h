@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define EP_ABI_VERSION 1
+#define EP_ABI_VERSION 2
 
 /* Exported symbols of libep_b200.so (everything else is hidden). */
 #if defined(__GNUC__)
@@ -82,7 +82,8 @@ enum {
  *   1 <= J <= 16, hidden >= 8 with hidden*2 a multiple of 16 bytes,
  *   expert_weight_elems >= 0 and a multiple of 8,
  *   R*S*ceil(expert_weight_elems/16) < 2^32, num_layers >= 1,
- *   0 <= waterfill_bonus_permille <= 1000.
+ *   0 <= waterfill_bonus_permille <= 1000, rerouting_mode in {0, 1},
+ *   solver_iter_limit >= 0.
  * Native placement is fixed: rank q hosts the contiguous block of experts
  * [q*(E/R) + min(q, E%R), ... + E/R + (q < E%R)) ([U] §"Shared redundant
  * slots": every logical expert keeps one fixed native instance).
@@ -104,7 +105,28 @@ typedef struct ep_config {
                                        ([W]'s all-rank mode) */
   int64_t expert_weight_elems;      /* Wn: bf16 elements of one expert (3*hidden*ffn) */
   uint64_t waterfill_seed;          /* seed of the per-token SplitMix64 draw */
+  uint64_t sampling_seed;           /* seed of the per-assignment draw of rerouting_mode 1 */
+  int32_t rerouting_mode;           /* EP_REROUTE_LOCAL_FIRST or EP_REROUTE_SAMPLED */
+  int32_t solver_iter_limit;        /* 0: the solver's bound 4(R*S + R + E) + 64; > 0: this
+                                       bound instead (drives EP_DEV_ITER_CAP in tests) */
 } ep_config;
+
+/* Rerouting modes (ep_config.rerouting_mode).  Both use the same quota solve.
+ * LOCAL_FIRST ([U] §"Quota"): each source rank's assignments of an expert use
+ * the instance on the source's own rank up to its quota, the rest fill the
+ * remote instances in instance order up to their remaining quotas; every
+ * instance receives exactly its quota.
+ * SAMPLED ([W] §"LPLB": the per-expert split, normalised to a distribution
+ * over the expert's physical instances, from which each token samples one):
+ * assignment a = (r*T + t)*K + k of expert e picks instance i of e with
+ * probability quota_i / total_e, drawn as h = SplitMix64(sampling_seed + a),
+ * u = ((h >> 32) * total_e) >> 32, i = first instance in instance order whose
+ * running quota sum exceeds u; an expert with one instance takes no draw.  An
+ * instance then receives as many rows as it drew (ep_layer_view.inst_count);
+ * rows inside an instance stay ordered by (source rank, t, k).  Waterfill's
+ * load score remains the solve's planned per-rank load. */
+#define EP_REROUTE_LOCAL_FIRST 0
+#define EP_REROUTE_SAMPLED 1
 
 /* Per-layer results, device-resident; copied to the host by ep_read_layer_stats. */
 typedef struct ep_layer_stats {
@@ -113,7 +135,8 @@ typedef struct ep_layer_stats {
   int32_t stop_reason;       /* EP_STOP_* of the chosen candidate */
   int32_t tight_stop_reason; /* EP_STOP_* of candidate j = 0 (the cap nearest the mean) */
   int32_t replicas;          /* replicas placed */
-  int32_t reserved0;
+  int32_t realized_max;      /* max per-rank routed rows actually dispatched: after_max,
+                                except in the sampled rerouting mode */
   int64_t cap;               /* cap C of the chosen candidate */
   int64_t assignments;       /* A: counted (valid) (token, k) assignments */
   int64_t rows;              /* dispatch rows: A, plus R*T with a shared expert */
@@ -147,6 +170,8 @@ typedef struct ep_layer_view {
                                    (ascending), instance order inside an expert */
   const int32_t* replica_expert_ptr; /* [E+1] CSR offsets of replica_list by expert */
   const ep_layer_stats* stats;  /* device copy of the layer's stats */
+  const int32_t* inst_count;    /* [R][G] rows each instance receives (inst_off's steps):
+                                   inst_quota itself except in the sampled rerouting mode */
   int32_t Gmax, G;              /* natives per rank (max) and columns per rank */
 } ep_layer_view;
 
@@ -275,6 +300,23 @@ EP_API ep_status_t ep_combine(ep_plan* plan, int32_t layer, const void* d_expert
 EP_API ep_status_t ep_waterfill(int32_t R, int32_t T, int32_t K, const int32_t* d_load,
                          const int32_t* d_dst_rank, uint64_t seed, int32_t bonus_permille,
                          int32_t flags, int32_t* d_pick, int32_t* d_count, void* stream);
+
+/*
+ * Waterfill re-run of a cached layer ([W] §"Waterfill"; [U] §"Reusing the
+ * forward plan": the layer's routed plan is kept and reused): re-draws every
+ * token's shared-expert rank of `layer` with `seed` in place of the plan's
+ * waterfill_seed — same candidates, waterline, slack, local preference and
+ * fallback as the pass inside ep_balance_layer, on the layer's routed rows and
+ * planned per-rank loads — and lays the shared columns out again.  Every rank's
+ * block keeps its routed rows in order; blocks shift with the new shared-column
+ * sizes, so the layer's dst_row, shared_rank, shared_row, the shared columns'
+ * inst_quota / inst_count, inst_off, rank_row_begin and stats.rows are all
+ * rewritten.  The result equals ep_balance_layer on the same ids with
+ * waterfill_seed = seed.  EP_ERR_UNSUPPORTED without a shared expert,
+ * EP_ERR_NOT_PLANNED before the layer's ep_balance_layer.  Uses the plan's
+ * scratch: must not overlap other calls on the plan.  Asynchronous on `stream`.
+ */
+EP_API ep_status_t ep_waterfill_layer(ep_plan* plan, int32_t layer, uint64_t seed, void* stream);
 
 /*
  * Load matrix without allocation.  The pages have no counterpart: this exists

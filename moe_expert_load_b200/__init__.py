@@ -11,6 +11,7 @@ the library is not built, importing the entry points raises (no fallback).
     plan.dispatch_tokens(0, hidden, out, 0, n)  # ep_dispatch_tokens (source-token range)
     plan.stage_replicas(0, native_w, slots)     # ep_stage_replicas
     plan.reduce_replica_grads(0, g_slots, g_native)
+    plan.waterfill_layer(0, seed)               # ep_waterfill_layer (shared expert)
 """
 from __future__ import annotations
 
@@ -74,6 +75,8 @@ def config_from_workload(w, num_layers: Optional[int] = None, **overrides) -> Ep
         waterfill_bonus_permille=w.waterfill_bonus_permille,
         waterfill_all_ranks=int(getattr(w, "waterfill_all_ranks", False)),
         expert_weight_elems=w.expert_elems, waterfill_seed=w.waterfill_seed,
+        sampling_seed=getattr(w, "sampling_seed", 0),
+        rerouting_mode=1 if getattr(w, "sampled_rerouting", False) else 0,
     )
     for k, v in overrides.items():
         setattr(c, k, v)
@@ -130,7 +133,7 @@ class Plan:
         rc = self.lib.ep_read_layer_stats(self.handle, layer, ctypes.byref(st), _stream(stream))
         if rc not in (EP_OK, EP_ERR_DEVICE_STATUS) or (raise_on_status and rc != EP_OK):
             raise EpError("ep_read_layer_stats", rc)
-        return {f: getattr(st, f) for f, _ in _abi.EpLayerStats._fields_ if f != "reserved0"}
+        return {f: getattr(st, f) for f, _ in _abi.EpLayerStats._fields_}
 
     def view(self, layer: int) -> dict:
         """ep_layer_view_get, returned as int32 tensors aliasing the workspace."""
@@ -142,7 +145,7 @@ class Plan:
             "inst_expert": (R, G), "inst_quota": (R, G), "inst_off": (R * G + 1,),
             "rank_row_begin": (R + 1,), "dst_row": (R, T, K), "shared_rank": (R, T),
             "shared_row": (R, T), "cand_max_load": (J,), "cand_replicas": (J,), "cand_stop": (J,),
-            "replica_list": (R * S,), "replica_expert_ptr": (E + 1,),
+            "replica_list": (R * S,), "replica_expert_ptr": (E + 1,), "inst_count": (R, G),
         }
         base = self.workspace.data_ptr()
         out = {"G": v.G, "Gmax": v.Gmax}
@@ -157,6 +160,11 @@ class Plan:
                 n *= s
             out[name] = self.workspace[off:off + 4 * n].view(torch.int32).view(shape)
         return out
+
+    def waterfill_layer(self, layer: int, seed: int, stream=None) -> None:
+        """ep_waterfill_layer: re-draw the layer's shared-expert ranks with `seed`."""
+        _check("ep_waterfill_layer", self.lib.ep_waterfill_layer(
+            self.handle, layer, ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), _stream(stream)))
 
     def dispatch_layout(self, layer: int, hidden: torch.Tensor, out: Optional[torch.Tensor] = None,
                         rank_begin: int = 0, rank_end: Optional[int] = None, out_rows: Optional[int] = None,

@@ -20,6 +20,9 @@ EP_DEV_WAIT_TIMEOUT = 4
 EP_DEV_OUT_CAPACITY = 8
 EP_DEV_INCONSISTENT = 16
 
+EP_REROUTE_LOCAL_FIRST = 0
+EP_REROUTE_SAMPLED = 1
+
 STOP_NAMES = {0: "BALANCED", 1: "SLOT_LIMITED", 2: "QUOTA_LIMITED", 3: "ITER_CAP"}
 
 # Every entry point include/ep_balance.h declares.
@@ -27,7 +30,7 @@ EXPORTS = (
     "ep_plan_workspace_bytes", "ep_plan_create", "ep_plan_destroy", "ep_balance_layer",
     "ep_layer_view_get", "ep_read_layer_stats", "ep_dispatch_layout", "ep_stage_replicas",
     "ep_reduce_replica_grads", "ep_waterfill", "ep_status_string", "ep_abi_version",
-    "ep_load_matrix_static", "ep_combine", "ep_dispatch_tokens",
+    "ep_load_matrix_static", "ep_combine", "ep_dispatch_tokens", "ep_waterfill_layer",
 )
 
 
@@ -40,6 +43,8 @@ class EpConfig(ctypes.Structure):
         ("num_cap_candidates", ctypes.c_int32), ("shared_expert", ctypes.c_int32),
         ("waterfill_bonus_permille", ctypes.c_int32), ("waterfill_all_ranks", ctypes.c_int32),
         ("expert_weight_elems", ctypes.c_int64), ("waterfill_seed", ctypes.c_uint64),
+        ("sampling_seed", ctypes.c_uint64), ("rerouting_mode", ctypes.c_int32),
+        ("solver_iter_limit", ctypes.c_int32),
     ]
 
 
@@ -47,7 +52,7 @@ class EpLayerStats(ctypes.Structure):
     _fields_ = [
         ("status", ctypes.c_int32), ("cap_idx", ctypes.c_int32),
         ("stop_reason", ctypes.c_int32), ("tight_stop_reason", ctypes.c_int32),
-        ("replicas", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+        ("replicas", ctypes.c_int32), ("realized_max", ctypes.c_int32),
         ("cap", ctypes.c_int64), ("assignments", ctypes.c_int64), ("rows", ctypes.c_int64),
         ("before_max", ctypes.c_int64), ("after_max", ctypes.c_int64),
     ]
@@ -56,7 +61,7 @@ class EpLayerStats(ctypes.Structure):
 _VIEW_PTRS = (
     "load", "expert_total", "rank_load_before", "rank_load", "inst_expert", "inst_quota",
     "inst_off", "rank_row_begin", "dst_row", "shared_rank", "shared_row", "cand_max_load",
-    "cand_replicas", "cand_stop", "replica_list", "replica_expert_ptr", "stats",
+    "cand_replicas", "cand_stop", "replica_list", "replica_expert_ptr", "stats", "inst_count",
 )
 
 
@@ -105,6 +110,7 @@ def load():
         "ep_reduce_replica_grads": (S, [P, I32, P, I32, P, P]),
         "ep_waterfill": (S, [I32, I32, I32, P, P, ctypes.c_uint64, I32, I32, P, P, P]),
         "ep_combine": (S, [P, I32, P, P, P, I32, P]),
+        "ep_waterfill_layer": (S, [P, I32, ctypes.c_uint64, P]),
         "ep_status_string": (ctypes.c_char_p, [S]),
         "ep_abi_version": (I32, []),
     }

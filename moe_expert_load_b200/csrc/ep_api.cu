@@ -24,11 +24,14 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
   // per layer (offset inside one layer block)
   size_t load, expert_total, W0, W, inst_expert, inst_quota, inst_off, rank_base, dst_row,
-      shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, stats;
+      shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, inst_count, stats;
   size_t layer_bytes;
   // scratch (absolute)
   size_t sub_cnt, blk_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase,
-      shared_tot, asg_rank, acc_load, acc_tot, acc_misc;
+      shared_tot, asg_rank, smp_cum, smp_inst, smp_key, smp_sub, smp_blk, smp_row0, rank_rows,
+      prev_base,
+      acc_load, acc_tot, acc_misc, smp_tot;
+  size_t acc_end;  // end of the accumulators zeroed before a plan's first balance call
   size_t scratch_bytes;
   size_t total;
 };
@@ -49,7 +52,9 @@ ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
       c->num_layers < 1 || c->num_cap_candidates < 1 || c->hidden < 1 ||
       c->expert_weight_elems < 0 || c->waterfill_bonus_permille < 0 ||
       (c->shared_expert != 0 && c->shared_expert != 1) ||
-      (c->waterfill_all_ranks != 0 && c->waterfill_all_ranks != 1))
+      (c->waterfill_all_ranks != 0 && c->waterfill_all_ranks != 1) ||
+      (c->rerouting_mode != EP_REROUTE_LOCAL_FIRST && c->rerouting_mode != EP_REROUTE_SAMPLED) ||
+      c->solver_iter_limit < 0)
     return EP_ERR_INVALID_ARGUMENT;
   const int Gmax = E / R + (E % R ? 1 : 0);
   if (R > ep::kMaxR || E > ep::kMaxE || Gmax > ep::kMaxNat || K > ep::kMaxK ||
@@ -80,6 +85,10 @@ ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
   d->hidden = c->hidden;
   d->seed = c->waterfill_seed;
   d->Wn = c->expert_weight_elems;
+  d->sampled = c->rerouting_mode == EP_REROUTE_SAMPLED;
+  d->iter_limit = c->solver_iter_limit;
+  d->sseed = c->sampling_seed;
+  d->nkey = E + R * d->S;  // at most 1024 + 128 * 8 keys: they fit the uint16 key buffer
   return EP_OK;
 }
 
@@ -104,6 +113,7 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.rep_eptr = b.take(i4 * (d.E + 1));
   L.rep_nexp = b.take(i4);
   L.rep_experts = b.take(i4 * ((size_t)d.R * d.S + 1));
+  L.inst_count = b.take(d.sampled ? i4 * d.R * d.G : 0);
   L.layer_bytes = b.off;
   Bump s;
   s.off = L.layer_bytes * (size_t)num_layers;
@@ -120,10 +130,22 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.sbase = s.take(i4 * d.R);
   L.shared_tot = s.take(i4 * d.R);
   L.asg_rank = s.take(d.sh ? (size_t)d.R * d.T * d.K : 0);
+  const size_t nblk = (d.nsub + ep::kPlanWarps - 1) / ep::kPlanWarps;
+  const size_t nk = d.sampled ? (size_t)d.nkey : 0;
+  L.smp_cum = s.take(i4 * nk);
+  L.smp_inst = s.take(i4 * nk);
+  L.smp_key = s.take(d.sampled ? sizeof(uint16_t) * (size_t)d.R * d.T * d.K : 0);
+  L.smp_sub = s.take(i4 * (size_t)d.R * d.nsub * nk);
+  L.smp_blk = s.take(i4 * (size_t)d.R * nblk * nk);
+  L.smp_row0 = s.take(i4 * (size_t)d.R * nk);
+  L.rank_rows = s.take(i4 * d.R);
+  L.prev_base = s.take(i4 * (d.R + 1));
   // contiguous: zeroed together once, before the plan's first balance call
   L.acc_load = s.take(i4 * (size_t)d.R * d.E);
   L.acc_tot = s.take(i4 * d.E);
   L.acc_misc = s.take(i4 * 4);
+  L.smp_tot = s.take(i4 * (size_t)d.R * nk);
+  L.acc_end = s.off;
   L.total = s.off;
   L.scratch_bytes = s.off - L.layer_bytes * (size_t)num_layers;
   return L;
@@ -169,6 +191,7 @@ ep::LayerBuf layer_buf(const ep_plan* p, int layer) {
   L.rep_eptr = at(p, b + l.rep_eptr);
   L.rep_nexp = at(p, b + l.rep_nexp);
   L.rep_experts = at(p, b + l.rep_experts);
+  L.inst_count = p->d.sampled ? at(p, b + l.inst_count) : L.inst_quota;
   L.stats = reinterpret_cast<ep_layer_stats*>(p->ws + b + l.stats);
   return L;
 }
@@ -192,6 +215,16 @@ ep::Scratch scratch(const ep_plan* p) {
   s.acc_load = at(p, l.acc_load);
   s.acc_tot = at(p, l.acc_tot);
   s.acc_misc = at(p, l.acc_misc);
+  const bool smp = p->d.sampled;
+  s.smp_tot = smp ? at(p, l.smp_tot) : nullptr;
+  s.smp_cum = smp ? at(p, l.smp_cum) : nullptr;
+  s.smp_inst = smp ? at(p, l.smp_inst) : nullptr;
+  s.smp_key = smp ? reinterpret_cast<uint16_t*>(p->ws + l.smp_key) : nullptr;
+  s.smp_sub = smp ? at(p, l.smp_sub) : nullptr;
+  s.smp_blk = smp ? at(p, l.smp_blk) : nullptr;
+  s.smp_row0 = smp ? at(p, l.smp_row0) : nullptr;
+  s.rank_rows = at(p, l.rank_rows);
+  s.prev_base = at(p, l.prev_base);
   return s;
 }
 
@@ -286,7 +319,7 @@ ep_status_t ep_balance_layer(ep_plan* plan, int32_t layer, const int32_t* d_topk
     // the workspace arrives uninitialised; after this every balance call
     // leaves the accumulators zero for the next
     const Layout& l = plan->lay;
-    const size_t bytes = l.acc_misc + 4 * sizeof(int32_t) - l.acc_load;
+    const size_t bytes = l.acc_end - l.acc_load;
     st = cuda_status(cudaMemsetAsync(plan->ws + l.acc_load, 0, bytes, s));
     if (st != EP_OK) return st;
     plan->acc_zero = true;
@@ -319,6 +352,7 @@ ep_status_t ep_layer_view_get(const ep_plan* plan, int32_t layer, ep_layer_view*
   out->replica_list = L.rep_list;
   out->replica_expert_ptr = L.rep_eptr;
   out->stats = L.stats;
+  out->inst_count = L.inst_count;
   out->Gmax = plan->d.Gmax;
   out->G = plan->d.G;
   return EP_OK;
@@ -426,6 +460,25 @@ ep_status_t ep_waterfill(int32_t R, int32_t T, int32_t K, const int32_t* d_load,
   return cuda_status(ep::launch_waterfill(R, T, K, d_load, d_dst_rank, seed, bonus_permille,
                                           flags & EP_WATERFILL_ALL_RANKS, d_pick, d_count,
                                           static_cast<cudaStream_t>(stream)));
+}
+
+ep_status_t ep_waterfill_layer(ep_plan* plan, int32_t layer, uint64_t seed, void* stream) {
+  ep_status_t st = check_layer(plan, layer);
+  if (st != EP_OK) return st;
+  if (!plan->d.sh) return EP_ERR_UNSUPPORTED;
+  if (!plan->planned[layer]) return EP_ERR_NOT_PLANNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!plan->acc_zero) {  // the shared scan's arrival ticket must start at zero
+    const Layout& l = plan->lay;
+    st = cuda_status(cudaMemsetAsync(plan->ws + l.acc_load, 0, l.acc_end - l.acc_load, s));
+    if (st != EP_OK) return st;
+    plan->acc_zero = true;
+  }
+  ep::Dims d = plan->d;
+  d.seed = seed;
+  st = cuda_status(ep::launch_waterfill_layer(d, layer_buf(plan, layer), scratch(plan), s));
+  if (st != EP_OK) plan->acc_zero = false;
+  return st;
 }
 
 }  // extern "C"

@@ -32,6 +32,10 @@ struct Dims {
   int all_ranks;     // Waterfill candidates: every rank
   uint64_t seed;     // Waterfill draw seed
   int64_t Wn;        // bf16 elements per expert
+  int sampled;       // rerouting mode: 1 = each assignment samples an instance
+  int iter_limit;    // > 0: the solver's iteration bound instead of 4(RS+R+E)+64
+  uint64_t sseed;    // seed of the sampled mode's per-assignment draw
+  int nkey;          // sampled mode: key space E + R*S (expert-major instance keys)
 };
 
 // One layer's slot in the plan cache (all device pointers).
@@ -52,6 +56,7 @@ struct LayerBuf {
   int32_t* rep_eptr;      // [E+1]
   int32_t* rep_nexp;      // [1] number of replicated experts
   int32_t* rep_experts;   // [R*S] replicated experts, ascending
+  int32_t* inst_count;    // [R][G] rows per instance (sampled mode; else inst_quota)
   ep_layer_stats* stats;
 };
 
@@ -76,6 +81,19 @@ struct Scratch {
   int32_t* acc_load;    // [R][E]
   int32_t* acc_tot;     // [E]
   int32_t* acc_misc;    // [0] status bits of the histogram, [1] arrival ticket
+  // Sampled rerouting mode only.  An instance key is kappa = e + rep_eptr[e] + j
+  // for the j-th instance of expert e in instance order (E + R*S keys at most).
+  int32_t* smp_tot;     // [R][nkey] draws per (source rank, key): an accumulator,
+                        // zero between calls like the ones above
+  int32_t* smp_cum;     // [nkey] running quota sum of the key's expert, inclusive
+  int32_t* smp_inst;    // [nkey] global instance index of the key
+  uint16_t* smp_key;    // [R][T][K] key drawn by each assignment (0xFFFF: dropped id)
+  int32_t* smp_sub;     // [R][nsub][nkey] draws per sub-chunk
+  int32_t* smp_blk;     // [R][ceil(nsub/kPlanWarps)][nkey] draws per block
+  int32_t* smp_row0;    // [R][nkey] first row of (source rank, key) (rank-relative
+                        // with a shared expert)
+  int32_t* rank_rows;   // [R] routed rows per destination rank
+  int32_t* prev_base;   // [R+1] a cached layer's rank bases before a Waterfill re-run
 };
 
 // ---- native placement: contiguous balanced blocks ---------------------------
@@ -115,6 +133,8 @@ cudaError_t launch_stage(const Dims& d, const LayerBuf& L, const void* native_w,
                          int num_sms, cudaStream_t st);
 cudaError_t launch_reduce(const Dims& d, const LayerBuf& L, void* slot_grads, int grad_f32,
                           float* native_grads, int num_sms, cudaStream_t st);
+cudaError_t launch_waterfill_layer(const Dims& d, const LayerBuf& L, const Scratch& s,
+                                   cudaStream_t st);
 cudaError_t launch_waterfill(int R, int T, int K, const int32_t* load, const int32_t* dst_rank,
                              uint64_t seed, int bonus, int all_ranks, int32_t* pick, int32_t* count,
                              cudaStream_t st);

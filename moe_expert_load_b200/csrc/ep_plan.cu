@@ -197,7 +197,6 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   if (tid == 0) {
     s_iter_cap_hit = 0;
     L.stats->status = s.acc_misc[0];  // the first status bits of this call
-    L.stats->reserved0 = 0;
     s.acc_misc[0] = 0;
   }
   __syncthreads();
@@ -245,7 +244,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       for (int t = 0; t < SMAX; ++t) { se[k][t] = -1; sq[k][t] = 0; }
     }
     __syncwarp();
-    const int iter_cap = 4 * (R * S + R + E) + 64;
+    const int iter_cap = d.iter_limit > 0 ? d.iter_limit : 4 * (R * S + R + E) + 64;
     // every key value is a load, a slack or a quota: at most C <= 1.08 A
     const bool pack = A < (1 << 24);
     for (int it = 0;; ++it) {
@@ -383,6 +382,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       if (q < R) {
         s_Wf[q] = Wr[k];
         L.W[q] = Wr[k];
+        s.rank_rows[q] = Wr[k];  // routed rows per rank (the sampled mode recounts them)
 #pragma unroll
         for (int t = 0; t < SMAX; ++t)
           if (t < S) { s_se[q * S + t] = se[k][t]; s_sq[q * S + t] = sq[k][t]; }
@@ -397,6 +397,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       st->cap = C;
       st->assignments = A;
       st->after_max = maxW;
+      st->realized_max = maxW;
       if (s_iter_cap_hit) atomicOr(&st->status, EP_DEV_ITER_CAP);
     }
   }
@@ -526,6 +527,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   __shared__ int32_t s_ipq[kWarpsPerBlock][kMaxR];    // instance j: start of residual interval
   __shared__ int32_t s_iloc[kWarpsPerBlock][kMaxR];   // instance j: local take
   __shared__ int32_t s_jof[kWarpsPerBlock][kMaxR];    // rank -> instance j or -1
+  __shared__ int32_t s_igi[kWarpsPerBlock][kMaxR];    // instance j: global instance index
   pdl_trigger();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -538,6 +540,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   int32_t* ipq = s_ipq[warp];
   int32_t* iloc = s_iloc[warp];
   int32_t* jof = s_jof[warp];
+  int32_t* igi = s_igi[warp];
 
   // the load column of e: independent of the instance lookups below, so its
   // loads are issued first
@@ -580,6 +583,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
       irel[j] = rel;
       iq[j] = quota;
       jof[q] = j;
+      igi[j] = q * G + col;
     }
     nrep += __popc(m);
     np += __popc(__ballot_sync(kFull, hit && q < h));
@@ -589,9 +593,32 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
     irel[np] = nat_rel;
     iq[np] = nat_q;
     jof[h] = np;
+    igi[np] = h * G + hcol;
   }
   const int ninst = nrep + 1;
   __syncwarp();
+  if (d.sampled) {
+    // the sampled mode needs, per instance key e + rep_eptr[e] + j, the running
+    // quota sum of e's instances in instance order and the instance's index
+    const int kb = e + L.rep_eptr[e];
+    int carry = 0;
+    for (int j0 = 0; j0 < ninst; j0 += 32) {
+      const int j = j0 + lane;
+      const int v = j < ninst ? iq[j] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (j < ninst) {
+        s.smp_cum[kb + j] = carry + incl;
+        s.smp_inst[kb + j] = igi[j];
+      }
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    return;
+  }
   // local take and residual demand of every source rank (lane owns r = lane + 32k)
   int Dr[kRW], locr[kRW];
 #pragma unroll
@@ -785,6 +812,53 @@ __device__ __forceinline__ int wf_pick(int r, int64_t token, const unsigned (&ma
     }
   }
   return W[r] <= W[lo] + B ? r : lo;
+}
+
+// a5 for one warp's sub-chunk of source rank r (tokens [t0, t1)): dr holds the
+// destination rank of each of the sub-chunk's assignments (kNoRank if none);
+// every token picks its shared-expert rank (wf_pick) and gets its ordinal among
+// the sub-chunk's tokens with the same pick (match.any groups, in token order);
+// the sub-chunk's pick counts per destination rank go to wsub_cnt for
+// k_shared_scan, and k_fixup turns the ordinals into rows.
+__device__ __forceinline__ void waterfill_subchunk(const Dims& d, const LayerBuf& L, const Scratch& s,
+                                                   int r, int sub, int t0, int t1,
+                                                   const uint8_t* dr, int32_t* wrun,
+                                                   const int32_t* s_slack, const int32_t* s_W,
+                                                   int lane) {
+  const int R = d.R, K = d.K;
+  const int gw = r * d.nsub + sub;
+  for (int q = lane; q < R; q += 32) wrun[q] = 0;
+  __syncwarp();
+  const int B = s.wf[1];
+  for (int t = t0; t < t1; t += 32) {
+    const int tt = t + lane;
+    int c = -1;
+    if (tt < t1) {
+      unsigned mask[kRW] = {0u, 0u, 0u, 0u};
+      if (d.all_ranks) {
+        mask_all(mask, R);
+      } else {
+        for (int k = 0; k < K; ++k) {
+          const int q = dr[(tt - t0) * K + k];
+          if (q != kNoRank) mask_set(mask, q);
+        }
+      }
+      mask_clear(mask, r);
+      c = wf_pick(r, (int64_t)r * d.T + tt, mask, s_slack, s_W, B, d.seed);
+    }
+    const unsigned peers = __match_any_sync(kFull, c);
+    const int rk = __popc(peers & lanemask_lt());
+    const int o = c >= 0 ? wrun[c] + rk : 0;
+    __syncwarp();
+    if (c >= 0 && lane == __ffs(peers) - 1) wrun[c] = o + __popc(peers);
+    __syncwarp();
+    if (tt < t1) {
+      L.shared_rank[(int64_t)r * d.T + tt] = c;
+      L.shared_row[(int64_t)r * d.T + tt] = o;  // ordinal inside (c, sub-chunk) for now
+    }
+  }
+  __syncwarp();
+  for (int q = lane; q < R; q += 32) s.wsub_cnt[(int64_t)q * R * d.nsub + gw] = wrun[q];
 }
 
 // ---------------------------------------------------------------------------
@@ -995,41 +1069,363 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     }
   }
   if (__any_sync(kFull, inconsistent) && lane == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
-  if (PASS > 0) {
-    const int gw = r * d.nsub + sub;
-    for (int q = lane; q < R; q += 32) wrun[q] = 0;
-    __syncwarp();
-    const int B = s.wf[1];
-    for (int t = t0; t < t1; t += 32) {
-      const int tt = t + lane;
-      int c = -1;
-      if (tt < t1) {
-        unsigned mask[kRW] = {0u, 0u, 0u, 0u};
-        if (d.all_ranks) {
-          mask_all(mask, R);
-        } else {
-          for (int k = 0; k < K; ++k) {
-            const int q = dr[(tt - t0) * K + k];
-            if (q != kNoRank) mask_set(mask, q);
-          }
-        }
-        mask_clear(mask, r);
-        c = wf_pick(r, (int64_t)r * d.T + tt, mask, s_slack, s_W, B, d.seed);
+  if (PASS > 0) waterfill_subchunk(d, L, s, r, sub, t0, t1, dr, wrun, s_slack, s_W, lane);
+}
+
+// ---------------------------------------------------------------------------
+// Sampled rerouting ("Waterfill and LPLB" page, section "LPLB": the per-expert
+// split, normalised to a distribution over the expert's physical instances,
+// from which every token samples one instance).  An instance key is
+// kappa = e + rep_eptr[e] + j for the j-th instance of e in instance order, so
+// the keys of one expert are contiguous and there are E + replicas of them.
+//
+// k_sample: same blocks as k_hist.  Each assignment a = (r*T + t)*K + k of
+// expert e draws its key: with more than one instance,
+// h = SplitMix64(sampling_seed + a), u = ((h >> 32) * total_e) >> 32 and the
+// key is the first of e's keys whose running quota sum exceeds u (binary
+// search); with one instance, that instance.  The warp counts its keys in a
+// shared histogram and writes the sub-chunk's row of counts; the block writes
+// its sum and adds it into the per-(source rank, key) accumulator.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+k_sample(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
+  extern __shared__ int32_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
+  const int E = d.E, K = d.K, NK = d.nkey;
+  const int nbpr = (d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const int r = blockIdx.x / nbpr, b = blockIdx.x - r * nbpr;
+  const int sub = b * kWarpsPerBlock + warp;
+  int32_t* s_cum = sm;                 // [NK]
+  int32_t* s_eptr = s_cum + NK;        // [E+1]
+  int32_t* s_tot = s_eptr + E + 1;     // [E]
+  int32_t* hists = s_tot + E;          // [warps][NK]
+  int32_t* hist = hists + warp * NK;
+  pdl_trigger();
+  pdl_wait();
+  for (int e = tid; e <= E; e += nthr) s_eptr[e] = L.rep_eptr[e];
+  for (int e = tid; e < E; e += nthr) s_tot[e] = L.expert_total[e];
+  __syncthreads();
+  const int nk = E + s_eptr[E];  // keys in use
+  for (int i = tid; i < nk; i += nthr) s_cum[i] = s.smp_cum[i];
+  for (int i = lane; i < nk; i += 32) hist[i] = 0;
+  __syncthreads();
+  if (sub < d.nsub) {
+    const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
+    const int64_t rbase = (int64_t)r * d.T * K;
+    const int a1 = t1 * K;
+    for (int a = t0 * K; a < a1; a += kBatch * 32) {
+      int v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = a + u * 32 + lane;
+        v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
       }
-      const unsigned peers = __match_any_sync(kFull, c);
-      const int rk = __popc(peers & lanemask_lt());
-      const int o = c >= 0 ? wrun[c] + rk : 0;
-      __syncwarp();
-      if (c >= 0 && lane == __ffs(peers) - 1) wrun[c] = o + __popc(peers);
-      __syncwarp();
-      if (tt < t1) {
-        L.shared_rank[(int64_t)r * d.T + tt] = c;
-        L.shared_row[(int64_t)r * d.T + tt] = o;  // ordinal inside (c, sub-chunk) for now
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int idx = a + u * 32 + lane;
+        if (idx >= a1) continue;
+        const int e = v[u];
+        int key = 0xFFFF;
+        if (e >= 0 && e < E) {
+          const int kb = e + s_eptr[e];
+          const int n = 1 + s_eptr[e + 1] - s_eptr[e];
+          int lo = 0;
+          if (n > 1) {
+            const uint64_t h = splitmix64(d.sseed + (uint64_t)(rbase + idx));
+            const int u32 = (int)(((h >> 32) * (uint64_t)s_tot[e]) >> 32);
+            int hi = n - 1;  // s_cum[kb + n - 1] = total > u: the answer exists
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (s_cum[kb + mid] > u32) hi = mid; else lo = mid + 1;
+            }
+          }
+          key = kb + lo;
+          atomicAdd(&hist[key], 1);
+        }
+        s.smp_key[rbase + idx] = (uint16_t)key;
       }
     }
     __syncwarp();
-    for (int q = lane; q < R; q += 32) s.wsub_cnt[(int64_t)q * R * d.nsub + gw] = wrun[q];
+    int32_t* out = s.smp_sub + ((int64_t)r * d.nsub + sub) * NK;
+    for (int i = lane; i < nk; i += 32) out[i] = hist[i];
   }
+  __syncthreads();
+  int32_t* blk = s.smp_blk + ((int64_t)r * nbpr + b) * NK;
+  for (int i = tid; i < nk; i += nthr) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarpsPerBlock; ++w) c += hists[w * NK + i];
+    blk[i] = c;
+    if (c) atomicAdd(&s.smp_tot[r * NK + i], c);
+  }
+}
+
+// k_sample_layout: one CTA.  Per key, the exclusive prefix of the draws over
+// source ranks (rows of earlier sources come first inside an instance) and
+// the key's total, which is its instance's row count; the accumulator is
+// zeroed for the next call.  Then the rank-relative first row of every
+// instance, each rank's routed rows, the dispatch layout (without a shared
+// expert; with one, k_shared_scan lays the ranks out) and the first row of
+// every (source rank, key), absolute or rank-relative.
+constexpr int kLayoutThreads = 1024;
+
+__global__ void __launch_bounds__(kLayoutThreads) k_sample_layout(Dims d, LayerBuf L, Scratch s) {
+  extern __shared__ int32_t sm[];
+  __shared__ int32_t s_base[kMaxR + 1];
+  __shared__ int32_t s_nk;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int R = d.R, E = d.E, G = d.G, NK = d.nkey, RG = d.R * d.G;
+  const int routed = d.Gmax + d.S;
+  int32_t* s_kcnt = sm;            // [NK] draws per key
+  int32_t* s_kinst = s_kcnt + NK;  // [NK] instance of the key
+  int32_t* s_icnt = s_kinst + NK;  // [R*G] rows per instance
+  int32_t* s_rel = s_icnt + RG;    // [R*G] rank-relative first row
+  pdl_trigger();
+  pdl_wait();
+  if (tid == 0) s_nk = E + L.rep_eptr[E];
+  for (int i = tid; i < RG; i += kLayoutThreads) s_icnt[i] = 0;
+  __syncthreads();
+  const int nk = s_nk;
+  for (int k = tid; k < nk; k += kLayoutThreads) {
+    int run = 0;
+    for (int r = 0; r < R; ++r) {
+      const int v = s.smp_tot[r * NK + k];
+      s.smp_tot[r * NK + k] = 0;  // zero again for the next call
+      s.smp_row0[r * NK + k] = run;
+      run += v;
+    }
+    s_kcnt[k] = run;
+    s_kinst[k] = s.smp_inst[k];
+  }
+  __syncthreads();
+  for (int k = tid; k < nk; k += kLayoutThreads) {
+    const int i = s_kinst[k];
+    if (i >= 0 && i < RG) s_icnt[i] = s_kcnt[k];  // each routed instance has one key
+  }
+  __syncthreads();
+  for (int i = tid; i < RG; i += kLayoutThreads) L.inst_count[i] = s_icnt[i];
+  if (tid < R) {
+    int run = 0;
+    for (int col = 0; col < G; ++col) {
+      s_rel[tid * G + col] = run;
+      s.inst_rel[tid * G + col] = run;
+      if (col < routed) run += s_icnt[tid * G + col];
+    }
+    s.rank_rows[tid] = run;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0, mx = 0;
+    for (int q0 = 0; q0 < R; q0 += 32) {
+      const int q = q0 + lane;
+      const int v = q < R ? s.rank_rows[q] : 0;
+      mx = max(mx, v);
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (q < R) s_base[q] = carry + incl - v;
+      carry += __shfl_sync(kFull, incl, 31);
+    }
+    mx = (int)__reduce_max_sync(kFull, (unsigned)mx);
+    if (lane == 0) {
+      s_base[R] = carry;
+      L.stats->realized_max = mx;
+    }
+  }
+  __syncthreads();
+  if (!d.sh) {
+    for (int i = tid; i < RG; i += kLayoutThreads) L.inst_off[i] = s_base[i / G] + s_rel[i];
+    if (tid == 0) {
+      L.inst_off[RG] = s_base[R];
+      L.stats->rows = s_base[R];
+    }
+    for (int q = tid; q <= R; q += kLayoutThreads) L.rank_base[q] = s_base[q];
+  }
+  for (int x = tid; x < R * nk; x += kLayoutThreads) {
+    const int r = x / nk, k = x - (x / nk) * nk;
+    const int i = s_kinst[k];
+    if (i < 0 || i >= RG) continue;
+    const int first = d.sh ? s_rel[i] : s_base[i / G] + s_rel[i];
+    s.smp_row0[r * NK + k] += first;
+  }
+}
+
+// k_sample_assign: same blocks as k_assign.  The row of an assignment with key
+// kappa is the first row of (r, kappa) plus its ordinal among rank r's
+// assignments with that key in (t, k) order: the counts of the rank's earlier
+// blocks and the block's earlier warps, the warp's running count and the rank
+// inside the 32-lane match.any group.  SH: rows relative to the destination
+// rank's block and the destination rank bytes, then the Waterfill picks
+// (waterfill_subchunk), exactly as k_assign<1>.
+template <int SH>
+__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+k_sample_assign(Dims d, LayerBuf L, Scratch s) {
+  extern __shared__ __align__(16) int32_t sm[];
+  __shared__ int32_t s_slack[kMaxR];
+  __shared__ int32_t s_W[kMaxR];
+  __shared__ int32_t s_nk;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
+  const int R = d.R, E = d.E, K = d.K, NK = d.nkey, G = d.G;
+  const int nbpr = (d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const int r = blockIdx.x / nbpr;
+  const int sub0 = (blockIdx.x - r * nbpr) * kWarpsPerBlock;
+  const int sub = sub0 + warp;
+  const bool active = sub < d.nsub;
+  int32_t* s_row0 = sm;                        // [NK] first row of (r, key)
+  int32_t* s_krank = s_row0 + NK;              // [NK] destination rank of the key (SH)
+  int32_t* base0 = s_krank + (SH ? NK : 0);    // [NK] draws of the rank's earlier blocks
+  const int per_warp = NK + (SH ? R + (kPlanSubT * K + 3) / 4 : 0);
+  int32_t* run = base0 + NK + warp * per_warp; // [NK] running ordinals
+  int32_t* wrun = run + NK;                    // [R] running shared ordinals (SH)
+  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);  // [kPlanSubT*K] ranks (SH)
+  pdl_trigger();
+  pdl_wait();
+  if (tid == 0) s_nk = E + L.rep_eptr[E];
+  __syncthreads();
+  const int nk = s_nk;
+  for (int k = tid; k < nk; k += nthr) {
+    s_row0[k] = s.smp_row0[r * NK + k];
+    if (SH) s_krank[k] = s.smp_inst[k] / G;
+    base0[k] = 0;
+  }
+  if (SH)
+    for (int q = tid; q < R; q += nthr) {
+      s_slack[q] = s.slack[q];
+      s_W[q] = L.W[q];
+    }
+  __syncthreads();
+  {
+    const int32_t* blk_r = s.smp_blk + (int64_t)r * nbpr * NK;
+    const int nb = sub0 / kWarpsPerBlock;
+    for (int b = 0; b < nb; ++b)
+      for (int k = tid; k < nk; k += nthr) base0[k] += blk_r[(int64_t)b * NK + k];
+  }
+  __syncthreads();
+  if (!active) return;
+  const int32_t* cnt_r = s.smp_sub + (int64_t)r * d.nsub * NK;
+  for (int k = lane; k < nk; k += 32) {
+    int acc = base0[k];
+    for (int w = 0; w < warp; ++w) acc += cnt_r[(int64_t)(sub0 + w) * NK + k];
+    run[k] = acc;
+  }
+  __syncwarp();
+  const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
+  const int a0 = t0 * K, a1 = t1 * K;
+  const int64_t rbase = (int64_t)r * d.T * K;
+  for (int a = a0; a < a1; a += kAsgBatch * 32) {
+    int v[kAsgBatch];
+#pragma unroll
+    for (int u = 0; u < kAsgBatch; ++u) {
+      const int idx = a + u * 32 + lane;
+      v[u] = idx < a1 ? (int)s.smp_key[rbase + idx] : 0xFFFF;
+    }
+#pragma unroll
+    for (int u = 0; u < kAsgBatch; ++u) {
+      if (a + u * 32 >= a1) break;
+      const int idx = a + u * 32 + lane;
+      const int key = v[u] < nk ? v[u] : -1;
+      const unsigned peers = __match_any_sync(kFull, key);
+      const int rk = __popc(peers & lanemask_lt());
+      const int o = key >= 0 ? run[key] + rk : 0;
+      __syncwarp();
+      if (key >= 0 && lane == __ffs(peers) - 1) run[key] = o + __popc(peers);
+      __syncwarp();
+      if (idx < a1) {
+        L.dst_row[rbase + idx] = key >= 0 ? s_row0[key] + o : -1;
+        if (SH) {
+          const uint8_t q = key >= 0 ? (uint8_t)s_krank[key] : (uint8_t)kNoRank;
+          dr[idx - a0] = q;
+          s.asg_rank[rbase + idx] = q;
+        }
+      }
+    }
+  }
+  if (SH) {
+    __syncwarp();
+    waterfill_subchunk(d, L, s, r, sub, t0, t1, dr, wrun, s_slack, s_W, lane);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Waterfill re-run of a cached layer.  k_wf_layer_prep (one CTA) rebuilds from
+// the layer's cache what the shared-slot pass reads from the scratch: routed
+// rows per rank and each instance's rank-relative first row (from the row
+// counts), the waterline H = ceil((A + N)/R), the local preference B and the
+// slack of every rank (from the planned loads), and keeps the old rank bases.
+// k_wf_layer (the blocks of k_assign) turns each routed row back into its
+// destination rank and rank-relative row, then draws the sub-chunk's shared
+// ranks (waterfill_subchunk); k_shared_scan and k_fixup lay the ranks out again.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_wf_layer_prep(Dims d, LayerBuf L, Scratch s) {
+  __shared__ int32_t s_A;
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const int R = d.R, G = d.G, routed = d.Gmax + d.S;
+  if (tid == 0) s_A = (int32_t)L.stats->assignments;
+  for (int q = tid; q <= R; q += blockDim.x) s.prev_base[q] = L.rank_base[q];
+  __syncthreads();
+  const int64_t N = (int64_t)R * d.T;
+  const int64_t H = ((int64_t)s_A + N + R - 1) / R;
+  if (tid == 0) {
+    s.wf[0] = (int)H;
+    s.wf[1] = (int)((H * d.bonus + 999) / 1000);
+  }
+  for (int q = tid; q < R; q += blockDim.x) {
+    int run = 0;
+    for (int col = 0; col < G; ++col) {
+      s.inst_rel[q * G + col] = run;
+      if (col < routed) run += L.inst_count[q * G + col];
+    }
+    s.rank_rows[q] = run;
+    s.slack[q] = (int)max(H - (int64_t)L.W[q], (int64_t)0);
+  }
+}
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) k_wf_layer(Dims d, LayerBuf L, Scratch s) {
+  extern __shared__ __align__(16) int32_t sm[];
+  __shared__ int32_t s_slack[kMaxR];
+  __shared__ int32_t s_W[kMaxR];
+  __shared__ int32_t s_pb[kMaxR + 1];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
+  const int R = d.R, K = d.K;
+  const int nbpr = (d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock;
+  const int r = blockIdx.x / nbpr;
+  const int sub = (blockIdx.x - r * nbpr) * kWarpsPerBlock + warp;
+  const int per_warp = R + (kPlanSubT * K + 3) / 4;
+  int32_t* wrun = sm + warp * per_warp;                 // [R]
+  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);   // [kPlanSubT*K]
+  pdl_trigger();
+  pdl_wait();
+  for (int q = tid; q < R; q += nthr) {
+    s_slack[q] = s.slack[q];
+    s_W[q] = L.W[q];
+  }
+  for (int q = tid; q <= R; q += nthr) s_pb[q] = s.prev_base[q];
+  __syncthreads();
+  if (sub >= d.nsub) return;
+  const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
+  const int a0 = t0 * K, a1 = t1 * K;
+  const int64_t rbase = (int64_t)r * d.T * K;
+  for (int idx = a0 + lane; idx < a1; idx += 32) {
+    const int row = L.dst_row[rbase + idx];
+    uint8_t q8 = (uint8_t)kNoRank;
+    if (row >= 0) {
+      int lo = 0, hi = R - 1;  // the last rank whose block starts at or before row
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_pb[mid] <= row) lo = mid; else hi = mid - 1;
+      }
+      q8 = (uint8_t)lo;
+      L.dst_row[rbase + idx] = row - s_pb[lo];
+    }
+    dr[idx - a0] = q8;
+    s.asg_rank[rbase + idx] = q8;
+  }
+  __syncwarp();
+  waterfill_subchunk(d, L, s, r, sub, t0, t1, dr, wrun, s_slack, s_W, lane);
 }
 
 // Shared-slot layout: block c scans destination rank c's pick counts over
@@ -1093,7 +1489,7 @@ __global__ void __launch_bounds__(kScanThreads) k_shared_scan(Dims d, LayerBuf L
     int carry = 0;
     for (int q0 = 0; q0 < R; q0 += 32) {
       const int q = q0 + lane;
-      const int v = q < R ? L.W[q] + s.shared_tot[q] : 0;
+      const int v = q < R ? s.rank_rows[q] + s.shared_tot[q] : 0;
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -1111,14 +1507,15 @@ __global__ void __launch_bounds__(kScanThreads) k_shared_scan(Dims d, LayerBuf L
     const int q = i / G, cc = i - (i / G) * G;
     if (cc == scol) {
       L.inst_quota[i] = s.shared_tot[q];
-      L.inst_off[i] = s_base[q] + L.W[q];
+      L.inst_count[i] = s.shared_tot[q];
+      L.inst_off[i] = s_base[q] + s.rank_rows[q];
     } else {
       L.inst_off[i] = s_base[q] + s.inst_rel[i];
     }
   }
   for (int q = tid; q <= R; q += kScanThreads) {
     L.rank_base[q] = s_base[q];
-    if (q < R) s.sbase[q] = s_base[q] + L.W[q];
+    if (q < R) s.sbase[q] = s_base[q] + s.rank_rows[q];
   }
   if (tid == 0) {
     L.inst_off[R * G] = s_base[R];
@@ -1216,6 +1613,20 @@ k_waterfill(int R, int T, int K, const int32_t* __restrict__ load,
   atomicAdd(&count[c], 1);
 }
 
+size_t sample_smem(const Dims& d) {
+  return sizeof(int32_t) * ((size_t)d.nkey * (1 + kWarpsPerBlock) + 2 * (size_t)d.E + 1);
+}
+size_t sample_layout_smem(const Dims& d) {
+  return sizeof(int32_t) * (2 * (size_t)d.nkey + 2 * (size_t)d.R * d.G);
+}
+size_t sample_assign_smem(const Dims& d) {
+  const size_t per_warp = d.nkey + (d.sh ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
+  return sizeof(int32_t) *
+         ((size_t)d.nkey * (d.sh ? 3 : 2) + (size_t)kWarpsPerBlock * per_warp);
+}
+size_t wf_layer_smem(const Dims& d) {
+  return sizeof(int32_t) * (size_t)kWarpsPerBlock * (d.R + (kPlanSubT * d.K + 3) / 4);
+}
 size_t solve_smem(const Dims& d) {
   return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + 2 * ((size_t)d.E + 1) + (size_t)d.R * d.G);
 }
@@ -1266,7 +1677,12 @@ cudaError_t set_plan_attributes(int max_smem) {
   if ((e = allow_solve<8>(max_smem)) != cudaSuccess) return e;
   if ((e = allow_max_dynamic_smem(k_hist, max_smem)) != cudaSuccess) return e;
   if ((e = allow_max_dynamic_smem(k_assign<0>, max_smem)) != cudaSuccess) return e;
-  return allow_max_dynamic_smem(k_assign<1>, max_smem);
+  if ((e = allow_max_dynamic_smem(k_assign<1>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_sample, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_sample_layout, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_sample_assign<0>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_wf_layer, max_smem)) != cudaSuccess) return e;
+  return allow_max_dynamic_smem(k_sample_assign<1>, max_smem);
 }
 
 template <int SMAX>
@@ -1287,6 +1703,9 @@ cudaError_t launch_solve(const Dims& d, const LayerBuf& L, const Scratch& s, cud
   return launch_solve_rw<8>(d, L, s, st);
 }
 
+cudaError_t launch_shared_layout(const Dims& d, const LayerBuf& L, const Scratch& s,
+                                 cudaStream_t st);
+
 cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, const int32_t* ids,
                            cudaStream_t st) {
   // the histogram is a plain launch (it reads the caller's ids at once); every
@@ -1304,21 +1723,52 @@ cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s, c
   err = launch_pdl(k_reroute, (unsigned)((d.E + kWarpsPerBlock - 1) / kWarpsPerBlock), bt, 0, st, d,
                    L, s);
   if (err != cudaSuccess) return err;
+  if (d.sampled) {
+    // sampled rerouting: draw keys, lay the instances out, then the rows
+    if (nblk > 0) err = launch_pdl(k_sample, nblk, bt, sample_smem(d), st, ids, d, L, s);
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(k_sample_layout, 1, kLayoutThreads, sample_layout_smem(d), st, d, L, s);
+    if (err != cudaSuccess) return err;
+    if (nblk > 0)
+      err = d.sh ? launch_pdl(k_sample_assign<1>, nblk, bt, sample_assign_smem(d), st, d, L, s)
+                 : launch_pdl(k_sample_assign<0>, nblk, bt, sample_assign_smem(d), st, d, L, s);
+    if (err != cudaSuccess) return err;
+  }
   if (!d.sh) {
-    if (nblk > 0) err = launch_pdl(k_assign<0>, nblk, bt, assign_smem(d, 0), st, ids, d, L, s);
+    if (!d.sampled && nblk > 0)
+      err = launch_pdl(k_assign<0>, nblk, bt, assign_smem(d, 0), st, ids, d, L, s);
   } else {
-    if (nblk > 0) err = launch_pdl(k_assign<1>, nblk, bt, assign_smem(d, 1), st, ids, d, L, s);
+    if (!d.sampled && nblk > 0)
+      err = launch_pdl(k_assign<1>, nblk, bt, assign_smem(d, 1), st, ids, d, L, s);
     if (err != cudaSuccess) return err;
-    err = launch_pdl(k_shared_scan, (unsigned)d.R, kScanThreads, 0, st, d, L, s);
-    if (err != cudaSuccess) return err;
-    const int64_t A4 = (int64_t)d.R * d.T * d.K / 4, N = (int64_t)d.R * d.T;
-    const int64_t work = A4 > N ? A4 : N;
-    const int64_t fblk = (work + kFixThreads - 1) / kFixThreads;
-    if (work > 0)
-      err = launch_pdl(k_fixup, (unsigned)(fblk < 2048 ? fblk : 2048), kFixThreads, 0, st, d, L, s);
+    err = launch_shared_layout(d, L, s, st);
   }
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
+}
+
+cudaError_t launch_shared_layout(const Dims& d, const LayerBuf& L, const Scratch& s,
+                                 cudaStream_t st) {
+  cudaError_t err = launch_pdl(k_shared_scan, (unsigned)d.R, kScanThreads, 0, st, d, L, s);
+  if (err != cudaSuccess) return err;
+  const int64_t A4 = (int64_t)d.R * d.T * d.K / 4, N = (int64_t)d.R * d.T;
+  const int64_t work = A4 > N ? A4 : N;
+  const int64_t fblk = (work + kFixThreads - 1) / kFixThreads;
+  if (work > 0)
+    err = launch_pdl(k_fixup, (unsigned)(fblk < 2048 ? fblk : 2048), kFixThreads, 0, st, d, L, s);
+  return err;
+}
+
+cudaError_t launch_waterfill_layer(const Dims& d, const LayerBuf& L, const Scratch& s,
+                                   cudaStream_t st) {
+  k_wf_layer_prep<<<1, 256, 0, st>>>(d, L, s);
+  cudaError_t err = cudaPeekAtLastError();
+  if (err != cudaSuccess) return err;
+  const unsigned nblk = (unsigned)(d.R * ((d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock));
+  if (nblk > 0)
+    err = launch_pdl(k_wf_layer, nblk, kWarpsPerBlock * 32, wf_layer_smem(d), st, d, L, s);
+  if (err != cudaSuccess) return err;
+  return launch_shared_layout(d, L, s, st);
 }
 
 cudaError_t launch_waterfill(int R, int T, int K, const int32_t* load, const int32_t* dst_rank,

@@ -74,6 +74,8 @@ def _load():
         lib.orc_permute.restype = None
         lib.orc_combine.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P]
         lib.orc_combine.restype = None
+        lib.orc_quota_solve.argtypes = [ctypes.c_int32] * 5 + [P, P, P]
+        lib.orc_quota_solve.restype = ctypes.c_int32
         lib.orc_eplb_plus.argtypes = [ctypes.c_int32] * 3 + [P, P, P, P]
         lib.orc_eplb_plus.restype = ctypes.c_int32
         lib.orc_stage.argtypes = [ctypes.c_int32] * 4 + [P, ctypes.c_int64, P, P]
@@ -239,6 +241,17 @@ def permute_range(p: Plan, hidden_rows: np.ndarray, n0: int, out: np.ndarray) ->
     dst = np.ascontiguousarray(p.dst_row.reshape(-1, p.K)[n0:n0 + n])
     srow = None if p.shared_row is None else np.ascontiguousarray(p.shared_row.reshape(-1)[n0:n0 + n])
     _load().orc_permute(n, p.K, hidden_rows.strides[0], _p(hidden_rows), _p(dst), _p(srow), _p(out))
+
+
+def quota_solve(Tot: np.ndarray, R: int, S: int, m: int, J: int = 16):
+    """The quota solve alone from per-expert totals: (W [R], max load, replicas)."""
+    Tot = np.ascontiguousarray(Tot, dtype=np.int64)
+    W = np.zeros(R, np.int64)
+    mx = ctypes.c_int64()
+    n = _load().orc_quota_solve(R, Tot.shape[0], S, m, J, _p(Tot), _p(W), ctypes.byref(mx))
+    if n < 0:
+        raise ValueError("oracle quota_solve rejected its arguments")
+    return W, int(mx.value), int(n)
 
 
 def eplb_plus(Tot: np.ndarray, R: int, S: int):

@@ -620,6 +620,64 @@ int orc_plan(const orc_cfg* c, const int32_t* ids, int64_t* L, int64_t* Tot, int
   return ORC_OK;
 }
 
+/* ---- O3 + O4 alone: the quota solve from the per-expert totals ---------- */
+/* The same greedy at the same cap candidates and the same selection as
+ * orc_plan, without the load matrix, the rerouting or the layout: what a
+ * solve-latency comparison with another replication rule times.  Writes the
+ * chosen candidate's per-rank loads W[R]; returns its replica count (or -1). */
+int32_t orc_quota_solve(int32_t R, int32_t E, int32_t S, int32_t m, int32_t J, const int64_t* Tot,
+                        int64_t* W, int64_t* max_out) {
+  if (R < 1 || E < 1 || S < 0 || m < 1 || J < 1) return -1;
+  orc_cfg c;
+  memset(&c, 0, sizeof c);
+  c.R = R; c.E = E; c.S = S; c.m = m; c.J = J; c.K = 1;
+  int64_t* W0 = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
+  int64_t A = 0;
+  for (int32_t e = 0; e < E; ++e) A += Tot[e];
+  for (int32_t q = 0; q < R; ++q) {
+    W0[q] = 0;
+    for (int32_t i = 0; i < nat_count(q, E, R); ++i) W0[q] += Tot[nat_first(q, E, R) + i];
+  }
+  greedy_state g, best;
+  char* stuck = (char*)malloc((size_t)R);
+  char* slotlim = (char*)malloc((size_t)R);
+  int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(orc_gmax(E, R) + 1));
+  greedy_state* gs[2] = {&g, &best};
+  for (int k = 0; k < 2; ++k) {
+    gs[k]->W = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
+    gs[k]->Qn = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
+    gs[k]->slot_e = (int32_t*)malloc(sizeof(int32_t) * (size_t)(R * S + 1));
+    gs[k]->slot_q = (int64_t*)malloc(sizeof(int64_t) * (size_t)(R * S + 1));
+    gs[k]->used = (int32_t*)malloc(sizeof(int32_t) * (size_t)R);
+  }
+  int32_t best_j = -1;
+  for (int32_t j = 0; j < J; ++j) {
+    const int64_t num = A * (200 + j), den = 200 * (int64_t)R;
+    greedy(&c, Tot, W0, (num + den - 1) / den, &g, stuck, slotlim, order);
+    if (best_j < 0 || g.maxW < best.maxW || (g.maxW == best.maxW && g.replicas < best.replicas)) {
+      greedy_state tmp = best;
+      best = g;
+      g = tmp;
+      best_j = j;
+    }
+  }
+  for (int32_t q = 0; q < R; ++q) W[q] = best.W[q];
+  *max_out = best.maxW;
+  const int32_t replicas = best.replicas;
+  for (int k = 0; k < 2; ++k) {
+    free(gs[k]->W);
+    free(gs[k]->Qn);
+    free(gs[k]->slot_e);
+    free(gs[k]->slot_q);
+    free(gs[k]->used);
+  }
+  free(W0);
+  free(stuck);
+  free(slotlim);
+  free(order);
+  return replicas;
+}
+
 /* ---- O10 standalone: Waterfill for given per-rank loads and routes ------ */
 /* load[R]: routed load per rank; dst_rank[R][T][K]: destination rank of each
  * routed assignment (-1 = none).  Writes pick[R][T] and count[R]. */

@@ -12,7 +12,8 @@ from moe_expert_load_b200 import Plan, config_from_workload
 def oracle_plan(w, ids, **kw):
     args = dict(E=w.E, S=w.S, m=w.m, J=w.J, shared_expert=w.shared_expert,
                 seed=w.waterfill_seed, bonus_permille=w.waterfill_bonus_permille,
-                all_ranks=w.waterfill_all_ranks)
+                all_ranks=w.waterfill_all_ranks, sampling=w.sampled_rerouting,
+                sampling_seed=w.sampling_seed)
     args.update(kw)
     return oracle.plan(ids, **args)
 
@@ -46,6 +47,7 @@ def compare_plan(g, o, w):
     np.testing.assert_array_equal(g["cand_stop"], o.cand_stop)
     np.testing.assert_array_equal(g["inst_expert"], o.inst_expert)
     np.testing.assert_array_equal(g["inst_quota"], o.inst_quota)
+    np.testing.assert_array_equal(g["inst_count"], o.inst_count)
     np.testing.assert_array_equal(g["inst_off"], o.inst_off)
     np.testing.assert_array_equal(g["dst_row"], o.dst_row)
     if o.shared_rank is not None:
@@ -64,6 +66,7 @@ def compare_plan(g, o, w):
     assert st["rows"] == o.rows
     assert st["before_max"] == o.before_max
     assert st["after_max"] == o.after_max
+    assert st["realized_max"] == o.realized_max
     # replica lists grouped by expert, instance order inside an expert
     S, Gm = o.S, o.Gmax
     ptr = g["replica_expert_ptr"]

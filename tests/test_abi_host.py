@@ -48,14 +48,14 @@ def test_only_declared_symbols_are_exported():
 
 
 def test_abi_version_and_strings():
-    assert ep_abi_version() == 1
+    assert ep_abi_version() == 2
     lib = _abi.load()
     assert lib.ep_status_string(2) == b"unsupported configuration"
 
 
 def test_struct_sizes_match_header():
-    # ep_config: 12 int32 + int64 + uint64; ep_layer_stats: 6 int32 + 5 int64
-    assert ctypes.sizeof(_abi.EpConfig) == 64
+    # ep_config: 12 int32 + int64 + 2 uint64 + 2 int32; ep_layer_stats: 6 int32 + 5 int64
+    assert ctypes.sizeof(_abi.EpConfig) == 80
     assert ctypes.sizeof(_abi.EpLayerStats) == 64
 
 
@@ -73,6 +73,7 @@ def test_workspace_sizes(name):
     ("slots_per_rank", 9, 2), ("num_cap_candidates", 17, 2), ("hidden", 12, 2),
     ("expert_weight_elems", 12, 2), ("min_replica_quota", 0, 1), ("waterfill_all_ranks", 2, 1),
     ("waterfill_bonus_permille", 1001, 2), ("shared_expert", 2, 1), ("tokens_per_rank", -1, 1),
+    ("rerouting_mode", 2, 1), ("solver_iter_limit", -1, 1),
 ])
 def test_config_validation(field, value, code):
     c = config_from_workload(get_config("tiny"))

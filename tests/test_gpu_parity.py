@@ -227,6 +227,87 @@ def test_plan_invariants_on_gpu_output():
     assert ratio <= 1.05 or g["stats"]["tight_stop_reason"] == 1
 
 
+# ---- sampled rerouting ("Waterfill and LPLB" page, section "LPLB") ---------------
+@pytest.mark.parametrize("name", ["tiny", "qwen", "dsv3", "stress"])
+def test_plan_parity_sampled_full_configs(name):
+    w = get_config(name).replace(sampled_rerouting=True)
+    ids = topk_ids(get_config(name))
+    o = oracle_plan(w, ids)
+    g = fetch(gpu_plan(w, ids))
+    compare_plan(g, o, w)
+    if o.replicas:
+        assert (o.inst_count != o.inst_quota).any()  # the draws are not the quotas
+
+
+def test_plan_parity_sampled_random_shapes():
+    rng = np.random.default_rng(777)
+    for case in range(30):
+        R, E, K, T, S, m, shared, J, ids = _random_case(rng)
+        if case % 3 == 0 and T:
+            ids[0, 0, 0] = E  # a dropped id
+        w = get_config("tiny").replace(R=R, E=E, K=K, T=T, S=S, m=m, J=J, shared_expert=shared,
+                                       sampled_rerouting=True, sampling_seed=int(rng.integers(0, 2**62)),
+                                       waterfill_all_ranks=bool(case % 2))
+        o = oracle_plan(w, ids)
+        compare_plan(fetch(gpu_plan(w, ids)), o, w)
+
+
+@pytest.mark.parametrize("R,E,K,T,S,shared", [
+    (128, 1024, 16, 40, 8, True),   # the largest key space: E + R*S = 2048 keys
+    (4, 128, 8, 600, 8, False),     # every slot filled
+])
+def test_plan_parity_sampled_maximum_shapes(R, E, K, T, S, shared):
+    rng = np.random.default_rng(R + E + S)
+    if R == 4:
+        logp = np.full(E, -8.0)
+        logp[:32] = 0.0
+        g = rng.gumbel(size=(R * T, E)) + logp
+        ids = np.argpartition(-g, K - 1, axis=1)[:, :K].reshape(R, T, K).astype(np.int32)
+    else:
+        ids = _skewed_topk(rng, R, T, E, K, 1.3)
+    w = get_config("tiny").replace(R=R, E=E, K=K, T=T, S=S, m=1, J=16, shared_expert=shared,
+                                   sampled_rerouting=True, sampling_seed=99)
+    o = oracle_plan(w, ids)
+    compare_plan(fetch(gpu_plan(w, ids)), o, w)
+
+
+def test_sampled_dispatch_matches_oracle():
+    w = get_config("tiny").replace(T=777, shared_expert=True, sampled_rerouting=True)
+    ids = topk_ids(get_config("tiny"))[:, :777].copy()
+    plan = gpu_plan(w, ids)
+    hidden = _hidden(w, 9)
+    out = plan.dispatch_layout(0, hidden)
+    torch.cuda.synchronize()
+    o = oracle_plan(w, ids)
+    want = oracle.permute(o, hidden.view(torch.int16).cpu().numpy())
+    np.testing.assert_array_equal(out.view(torch.int16).cpu().numpy()[: o.rows], want)
+    assert plan.read_layer_stats(0)["status"] == 0
+
+
+# ---- the solver's iteration bound -------------------------------------------------
+@pytest.mark.parametrize("name,limit", [("qwen", 2), ("dsv3", 5), ("tiny", 1)])
+def test_iteration_bound_sets_status_and_keeps_a_valid_plan(name, limit):
+    # a bound smaller than the moves the greedy needs: every candidate stops
+    # there, the status bit is set and the plan is still a valid layout equal
+    # to the oracle's under the same bound
+    w = get_config(name)
+    ids = topk_ids(w)
+    o = oracle_plan(w, ids, iter_limit=limit)
+    assert o.status & oracle.ST_ITER_CAP
+    plan = gpu_plan(w, ids, solver_iter_limit=limit)
+    g = fetch(plan)
+    compare_plan(g, o, w)
+    assert g["stats"]["status"] & 2  # EP_DEV_ITER_CAP
+    assert (g["cand_stop"] == 3).any()
+    check_plan(ids, w.E, w.S, w.m, Gmax=g["Gmax"], G=g["G"], W=g["rank_load"],
+               inst_expert=g["inst_expert"], inst_quota=g["inst_quota"], inst_off=g["inst_off"],
+               dst_row=g["dst_row"], cap=g["stats"]["cap"], shared_rank=g["shared_rank"],
+               shared_row=g["shared_row"])
+    # the next call without the bound (another plan, same ids) is clean
+    assert plan.read_layer_stats(0)["status"] & 2
+    assert fetch(gpu_plan(w, ids))["stats"]["status"] == 0
+
+
 # ---- dispatch permutation ------------------------------------------------------
 def _hidden(w, seed=0):
     g = torch.Generator(device="cuda")
@@ -268,6 +349,74 @@ def test_dispatch_full_qwen_round_trip():
     dst = plan.view(0)["dst_row"].reshape(w.N, w.K).long()
     for k in range(w.K):  # gather back by dst_row: bitwise the source rows
         assert torch.equal(out[dst[:, k]].view(torch.int16), hidden.view(torch.int16))
+    assert plan.read_layer_stats(0)["status"] == 0
+
+
+def _rows_hold_tokens(out, lo, hi, rows_np, hidden, chunk=1 << 15):
+    """out[row - lo] == hidden[n] (bitwise) for every token n whose oracle row
+    `rows_np[n]` lies in [lo, hi); returns how many rows were checked."""
+    n_all = np.nonzero((rows_np >= lo) & (rows_np < hi))[0]
+    for a in range(0, len(n_all), chunk):
+        n = torch.from_numpy(n_all[a:a + chunk]).cuda()
+        r = torch.from_numpy(rows_np[n_all[a:a + chunk]] - lo).cuda()
+        assert torch.equal(out[r].view(torch.int16), hidden[n].view(torch.int16))
+    return len(n_all)
+
+
+def _count_unwritten(out, sentinel=-1, chunk=1 << 16):
+    bad = 0
+    o16 = out.view(torch.int16)
+    for a in range(0, o16.shape[0], chunk):
+        bad += int((o16[a:a + chunk] == sentinel).all(dim=1).sum())
+    return bad
+
+
+def test_dispatch_dsv3_full_matches_oracle_rows():
+    # the whole DeepSeek-V3-shaped layer (routed and shared rows, 33.8 GB):
+    # every token's row, at the position the oracle's layout gives it, holds
+    # the token's hidden state, and no row is left unwritten
+    w = get_config("dsv3")
+    ids = topk_ids(w)
+    o = oracle_plan(w, ids)
+    plan = gpu_plan(w, ids)
+    hidden = _hidden(w, 6)
+    out = torch.full((o.rows, w.hidden), -1, dtype=torch.int16, device="cuda")
+    plan.dispatch_layout(0, hidden, out=out.view(torch.bfloat16))
+    torch.cuda.synchronize()
+    dst = o.dst_row.reshape(w.N, w.K)
+    checked = sum(_rows_hold_tokens(out, 0, o.rows, np.ascontiguousarray(dst[:, k]), hidden)
+                  for k in range(w.K))
+    checked += _rows_hold_tokens(out, 0, o.rows, o.shared_row.reshape(w.N), hidden)
+    assert checked == o.rows == w.A + w.N
+    assert _count_unwritten(out) == 0
+    assert plan.read_layer_stats(0)["status"] == 0
+
+
+def test_dispatch_stress_rank_windows_match_oracle_rows():
+    # the stress layer's 135 GB layout does not fit one GPU next to its input:
+    # it is dispatched in destination-rank windows; each window holds exactly
+    # the oracle's rows of those ranks
+    w = get_config("stress")
+    ids = topk_ids(w)
+    o = oracle_plan(w, ids)
+    plan = gpu_plan(w, ids)
+    hidden = _hidden(w, 7)
+    rb = o.inst_off[np.arange(w.R + 1) * o.G]
+    dst = o.dst_row.reshape(w.N, w.K)
+    cols = [np.ascontiguousarray(dst[:, k]) for k in range(w.K)]
+    total = 0
+    for b, e in [(0, 18), (18, 37), (37, 72)]:
+        lo, hi = int(rb[b]), int(rb[e])
+        out = torch.full((hi - lo, w.hidden), -1, dtype=torch.int16, device="cuda")
+        plan.dispatch_layout(0, hidden, out=out.view(torch.bfloat16), rank_begin=b, rank_end=e)
+        torch.cuda.synchronize()
+        checked = sum(_rows_hold_tokens(out, lo, hi, c, hidden) for c in cols)
+        assert checked == hi - lo
+        assert _count_unwritten(out) == 0
+        total += checked
+        del out
+        torch.cuda.empty_cache()
+    assert total == o.rows == w.A
     assert plan.read_layer_stats(0)["status"] == 0
 
 
@@ -383,9 +532,12 @@ def test_dispatch_capacity_overflow_is_flagged_not_written():
 
 # ---- replica staging and gradient reduction -----------------------------------
 def test_stage_replicas_qwen():
+    # which expert each slot must hold comes from the oracle's plan, not from
+    # the plan under test
     w = get_config("qwen")
     ids = topk_ids(w)
     plan = gpu_plan(w, ids)
+    o = oracle_plan(w, ids)
     Wn = w.expert_elems
     g = torch.Generator(device="cuda")
     g.manual_seed(5)
@@ -393,19 +545,16 @@ def test_stage_replicas_qwen():
     slots = torch.full((w.R, w.S, Wn), 7, dtype=torch.int16, device="cuda")
     plan.stage_replicas(0, native.view(torch.bfloat16), slots.view(torch.bfloat16))
     torch.cuda.synchronize()
-    v = plan.view(0)
-    ie = v["inst_expert"].cpu().numpy()
-    Gm = v["Gmax"]
     filled = 0
     for q in range(w.R):
         for s in range(w.S):
-            e = int(ie[q, Gm + s])
+            e = int(o.inst_expert[q, o.Gmax + s])
             if e >= 0:
                 filled += 1
                 assert torch.equal(slots[q, s], native[e])
             else:
                 assert bool((slots[q, s] == 7).all())
-    assert filled == plan.read_layer_stats(0)["replicas"] > 0
+    assert filled == o.replicas == plan.read_layer_stats(0)["replicas"] > 0
 
 
 @pytest.mark.parametrize("grad_dtype", ["bf16", "f32"])
@@ -452,6 +601,46 @@ def test_waterfill_standalone_parity(all_ranks):
             wp, wc = oracle.waterfill(load, dst, seed=seed, bonus_permille=bonus, all_ranks=all_ranks)
             np.testing.assert_array_equal(pick.cpu().numpy(), wp)
             np.testing.assert_array_equal(count.cpu().numpy(), wc)
+
+
+@pytest.mark.parametrize("name,all_ranks,sampled", [
+    ("dsv3", False, False), ("tiny", True, False), ("dsv3", False, True)])
+def test_waterfill_layer_rerun_equals_a_fresh_balance(name, all_ranks, sampled):
+    # a cached layer re-drawn with another seed equals the oracle's plan of the
+    # same ids with that seed; another layer balanced in between (it rewrites
+    # the plan's scratch) does not matter
+    w0 = get_config(name).replace(shared_expert=True, waterfill_all_ranks=all_ranks,
+                                  sampled_rerouting=sampled)
+    ids = topk_ids(get_config(name))
+    other = np.ascontiguousarray(ids[::-1])
+    plan = Plan(config_from_workload(w0, num_layers=2))
+    gpu_plan(w0, ids, plan=plan, layer=0)
+    gpu_plan(w0, other, plan=plan, layer=1)
+    for seed in (12345, 2**64 - 3):
+        plan.waterfill_layer(0, seed)
+        torch.cuda.synchronize()
+        w1 = w0.replace(waterfill_seed=seed)
+        compare_plan(fetch(plan, 0), oracle_plan(w1, ids), w1)
+    compare_plan(fetch(plan, 1), oracle_plan(w0, other), w0)  # untouched
+    plan.waterfill_layer(0, w0.waterfill_seed)  # back to the plan's own seed
+    torch.cuda.synchronize()
+    compare_plan(fetch(plan, 0), oracle_plan(w0, ids), w0)
+
+
+def test_waterfill_layer_errors():
+    w = get_config("tiny")
+    plan = Plan(config_from_workload(w))
+    with pytest.raises(EpError) as ei:
+        plan.waterfill_layer(0, 1)
+    assert ei.value.status == 2  # no shared expert
+    ws = w.replace(shared_expert=True)
+    plan = Plan(config_from_workload(ws, num_layers=2))
+    with pytest.raises(EpError) as ei:
+        plan.waterfill_layer(0, 1)
+    assert ei.value.status == 5  # not balanced yet
+    with pytest.raises(EpError) as ei:
+        plan.waterfill_layer(2, 1)
+    assert ei.value.status == 1
 
 
 def test_plan_parity_waterfill_all_ranks():
@@ -523,11 +712,13 @@ def test_combine_matches_oracle(name, shared, out_dtype, sample):
     dt = torch.float32 if out_dtype == "f32" else torch.bfloat16
     y = plan.combine(0, x, wts, out_dtype=dt)
     torch.cuda.synchronize()
-    v = plan.view(0)
+    # the rows each token's terms come from: the oracle's layout
+    o = oracle_plan(w_cfg, ids)
+    assert o.rows == rows
     N = w_cfg.N
     toks = np.arange(N) if sample is None else np.random.default_rng(5).choice(N, sample, replace=False)
-    dst = v["dst_row"].reshape(N, w_cfg.K).cpu().numpy()[toks]
-    srow = None if not shared else v["shared_row"].reshape(N).cpu().numpy()[toks]
+    dst = o.dst_row.reshape(N, w_cfg.K)[toks]
+    srow = None if not shared else o.shared_row.reshape(N)[toks]
     xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
     wn = wts.reshape(N, w_cfg.K).cpu().numpy()[toks]
     want = oracle.combine_tokens(xb, dst, wn, srow)

@@ -749,3 +749,13 @@ def test_iteration_limit_stops_the_greedy_and_keeps_a_valid_plan():
     assert (p.cand_repl <= 2).all()
     assert p.stop_name == "ITER_CAP"
     _check(p, ids, cfg.E, cfg.S, cfg.m)
+
+
+@pytest.mark.parametrize("name", ["qwen", "dsv3"])
+def test_quota_solve_alone_matches_the_plan(name):
+    # the solve-latency comparison times the same solve the plan runs
+    cfg = get_config(name)
+    p = _plan_cfg(cfg, topk_ids(cfg))
+    W, mx, rep = oracle.quota_solve(p.Tot, cfg.R, cfg.S, cfg.m, cfg.J)
+    np.testing.assert_array_equal(W, p.W)
+    assert (mx, rep) == (p.after_max, p.replicas)

@@ -32,6 +32,8 @@ class WorkloadConfig:
     waterfill_seed: int = 0x5EED_0F_1A7E12
     waterfill_bonus_permille: int = 10
     waterfill_all_ranks: bool = False  # Waterfill candidates: all ranks instead of visited ones
+    sampled_rerouting: bool = False  # tokens sample an instance with probability quota/total
+    sampling_seed: int = 0x5A3B_1E5EED
 
     @property
     def N(self) -> int:

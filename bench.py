@@ -250,6 +250,10 @@ def run_gpu(args):
 
     world, rank, local = _dist_init()
     torch.cuda.set_device(local)
+    if args.dispatch_impl == "bulk":  # read by the library at plan creation
+        os.environ["EP_DISPATCH_IMPL"] = "bulk"
+    else:
+        os.environ.pop("EP_DISPATCH_IMPL", None)
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -407,7 +411,7 @@ def run_gpu(args):
     peak, peak_kind = _peaks()
     perm_bytes = (w.N + rows_cap) * w.hidden * 2  # each token row read once, written per row
     achieved = perm_bytes / (perm_avg_ms * 1e-3) / 1e9
-    traffic = _traffic("k_permute", w.name)
+    traffic = _traffic("k_permute", w.name) if args.dispatch_impl == "regs" else None
     A = int(stats["assignments"])
     line = {
         "metric": METRIC,
@@ -433,7 +437,9 @@ def run_gpu(args):
         "reduce_gbs": reduce_bytes / (reduce_ms * 1e-3) / 1e9 if n_rep else 0.0,
         "combine_gbs": combine_bytes / (combine_ms * 1e-3) / 1e9,
         "max_mean_load": _ratio(stats, w.R),
-        "roofline": {"bound": "hbm", "kernel": "k_permute", "achieved": achieved, "peak": peak,
+        "dispatch_impl": args.dispatch_impl,
+        "roofline": {"bound": "hbm", "kernel": "k_permute" if args.dispatch_impl == "regs"
+                     else "k_permute_bulk", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes": perm_bytes,
                      "launch_ms": perm_avg_ms},
@@ -699,6 +705,9 @@ def main():
     ap.add_argument("--tokens-per-rank", type=int, default=None,
                     help="override T (small cases for profiler captures)")
     ap.add_argument("--ffn", type=int, default=None, help="override the expert FFN width")
+    ap.add_argument("--dispatch-impl", default="regs", choices=["regs", "bulk"],
+                    help="dispatch kernel: register-staged (default) or the bulk-copy (TMA) "
+                         "variant, for comparing the two")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "cuda":
         ap.error("--warmup must be at least 3")

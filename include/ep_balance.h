@@ -182,7 +182,18 @@ typedef struct ep_plan ep_plan; /* opaque */
 EP_API ep_status_t ep_plan_workspace_bytes(const ep_config* cfg, size_t* bytes);
 
 /* Create a plan over caller-owned device workspace `d_workspace` (>= the size
- * above, 256-byte aligned).  Uses the current CUDA device.  Writes *out. */
+ * above, 256-byte aligned).  Uses the current CUDA device.  Writes *out.
+ * The copy kernels (dispatch, combine, staging, reduction) size their grids
+ * by the device's SM count; if the environment variable EP_GRID_SMS holds an
+ * integer in [1, 4096] when the plan is created, that count is used instead.
+ * No result depends on it (every output element is written by one thread of
+ * a grid-stride loop); it exists to test exactly that.
+ * If EP_DISPATCH_IMPL is "bulk" when the plan is created, ep_dispatch_layout
+ * and ep_dispatch_tokens move the rows with the bulk-copy (TMA) engine through
+ * a ring of shared-memory row buffers instead of staging them in registers
+ * (same results; measured slower on B200, kept to reproduce that
+ * measurement).  It falls back to the register path when four rows do not
+ * fit in shared memory or K + 1 > 32. */
 EP_API ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t workspace_bytes,
                            ep_plan** out);
 

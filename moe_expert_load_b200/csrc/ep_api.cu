@@ -3,6 +3,7 @@
 // entry points, each of which only validates arguments and enqueues kernels.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <new>
@@ -163,6 +164,7 @@ struct ep_plan {
   size_t ws_bytes;
   int device;
   int num_sms;
+  int dispatch_bulk;       // EP_DISPATCH_IMPL=bulk: the bulk-copy (TMA) dispatch variant
   unsigned char* planned;  // per layer: balanced at least once
   bool acc_zero;           // the scratch accumulators are known to be zero
 };
@@ -278,6 +280,12 @@ ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t works
   if (cudaGetDevice(&dev) != cudaSuccess) return EP_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return EP_ERR_CUDA;
+  // EP_GRID_SMS replaces the SM count the copy kernels size their grids by
+  // (results never depend on it; tests use it to check exactly that)
+  if (const char* env = getenv("EP_GRID_SMS")) {
+    const long v = strtol(env, nullptr, 10);
+    if (v > 0 && v <= 4096) sms = (int)v;
+  }
   int max_smem = 0;
   if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return EP_ERR_CUDA;
@@ -298,6 +306,10 @@ ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t works
   p->ws_bytes = workspace_bytes;
   p->device = dev;
   p->num_sms = sms;
+  {
+    const char* impl = getenv("EP_DISPATCH_IMPL");
+    p->dispatch_bulk = impl && strcmp(impl, "bulk") == 0;
+  }
   p->acc_zero = false;
   *out = p;
   return EP_OK;
@@ -388,7 +400,7 @@ ep_status_t ep_dispatch_layout(ep_plan* plan, int32_t layer, const void* d_hidde
   return cuda_status(ep::launch_dispatch(plan->d, layer_buf(plan, layer), d_hidden, d_out,
                                          out_rows_capacity, dst_rank_begin, dst_rank_end, 0,
                                          (int64_t)plan->d.R * plan->d.T, plan->num_sms,
-                                         static_cast<cudaStream_t>(stream)));
+                                         plan->dispatch_bulk, static_cast<cudaStream_t>(stream)));
 }
 
 ep_status_t ep_dispatch_tokens(ep_plan* plan, int32_t layer, const void* d_hidden, int64_t token_begin,
@@ -404,7 +416,8 @@ ep_status_t ep_dispatch_tokens(ep_plan* plan, int32_t layer, const void* d_hidde
   if (!d_hidden || !d_out || !aligned16(d_hidden) || !aligned16(d_out)) return EP_ERR_INVALID_ARGUMENT;
   return cuda_status(ep::launch_dispatch(plan->d, layer_buf(plan, layer), d_hidden, d_out,
                                          out_rows_capacity, 0, plan->d.R, token_begin, token_end,
-                                         plan->num_sms, static_cast<cudaStream_t>(stream)));
+                                         plan->num_sms, plan->dispatch_bulk,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 ep_status_t ep_combine(ep_plan* plan, int32_t layer, const void* d_expert_out, const float* d_weights,

@@ -134,6 +134,158 @@ __global__ void __launch_bounds__(kPermuteThreads) k_permute(PermuteArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// a6, bulk-copy variant (EP_DISPATCH_IMPL=bulk at plan creation): the same
+// permutation moved by the bulk-copy (TMA) engine instead of registers.  One
+// warp per CTA keeps a ring of NST row buffers in shared memory; lane 0 loads
+// token j's row with cp.async.bulk (completion counted on the stage's
+// mbarrier) LA tokens ahead of storing it, and stores each kept row with
+// cp.async.bulk from shared memory, one bulk group per token; a stage is
+// reused once the group that last read it has finished reading (NST - LA
+// groups of slack).  Loads carry no multicast.  Every mbarrier wait is
+// bounded: on timeout the kernel flags EP_DEV_WAIT_TIMEOUT, stops issuing,
+// waits (bounded) for the loads it has in flight and returns.
+// ---------------------------------------------------------------------------
+constexpr int kBulkStages = 4;      // row buffers per CTA
+constexpr int kBulkAhead = 2;       // tokens loaded ahead of the one being stored
+constexpr uint32_t kBulkSpinLimit = 1u << 22;  // polls of one mbarrier before giving up
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait for the phase with the given parity; false on timeout
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kBulkSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst_smem)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_addr(src_smem)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+template <int NST, int LA>
+__global__ void __launch_bounds__(32) k_permute_bulk(PermuteArgs a) {
+  static_assert(LA >= 1 && LA < NST, "stores need slack behind the loads");
+  extern __shared__ __align__(128) uint8_t bbuf[];
+  __shared__ __align__(8) uint64_t bar[NST];
+  __shared__ int32_t sd[NST][kMaxK + 1];
+  __shared__ uint32_t smask[NST];
+  const int lane = threadIdx.x;
+  const uint32_t row_bytes = (uint32_t)a.row16 * 16u;
+  const int row_lo = a.rank_base[a.rank_begin];
+  const int row_hi = a.rank_base[a.rank_end];
+  const uint8_t* hidden = reinterpret_cast<const uint8_t*>(a.hidden);
+  uint8_t* out = reinterpret_cast<uint8_t*>(a.out);
+  if (lane == 0) {
+    for (int st = 0; st < NST; ++st) mbar_init(&bar[st], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const int64_t first = a.n0 + blockIdx.x;
+  const int64_t count = first < a.N ? (a.N - first + gridDim.x - 1) / gridDim.x : 0;
+  uint32_t phase = 0, inflight = 0;  // lane 0: per-stage parity and loads in flight
+  bool overflow = false, timeout = false;
+  for (int64_t j = 0; j < count + LA; ++j) {
+    // store token j - LA: wait for its row, then one bulk store per kept row
+    const int64_t js = j - LA;
+    if (js >= 0 && lane == 0) {
+      const int st = (int)(js % NST);
+      const uint32_t m = smask[st];
+      if (m) {
+        if (mbar_wait(&bar[st], (phase >> st) & 1u)) {
+          phase ^= 1u << st;
+          inflight &= ~(1u << st);
+          uint32_t mm = m;
+          while (mm) {
+            const int from = __ffs(mm) - 1;
+            mm &= mm - 1;
+            bulk_store(out + (int64_t)sd[st][from] * row_bytes, bbuf + (size_t)st * row_bytes,
+                       row_bytes);
+          }
+        } else {
+          timeout = true;
+        }
+      }
+      bulk_commit();  // one group per token, possibly empty
+    }
+    timeout = __shfl_sync(kFull, timeout ? 1 : 0, 0) != 0;
+    if (timeout) break;  // the same on every lane
+    // issue token j into stage j % NST
+    if (j < count) {
+      const int st = (int)(j % NST);
+      const int64_t n = first + j * gridDim.x;
+      int d = -1;
+      if (lane < a.K) d = a.dst_row[n * a.K + lane];
+      else if (lane == a.K && a.shared_row != nullptr) d = a.shared_row[n];
+      d = (d >= row_lo && d < row_hi) ? d - row_lo : -1;
+      if (d >= a.cap_rows) {
+        overflow = true;
+        d = -1;
+      }
+      const unsigned m = __ballot_sync(kFull, d >= 0);
+      // the stage's previous token, j - NST, was stored NST - LA iterations ago:
+      // once at most NST - LA newer groups are pending, its group has
+      // finished reading the buffer
+      if (lane == 0) bulk_wait_read<NST - LA>();
+      __syncwarp();
+      if (lane <= a.K) sd[st][lane] = d;
+      if (lane == 0) {
+        smask[st] = m;
+        if (m) {
+          mbar_expect_tx(&bar[st], row_bytes);
+          bulk_load(bbuf + (size_t)st * row_bytes, hidden + n * (int64_t)row_bytes, row_bytes,
+                    &bar[st]);
+          inflight |= 1u << st;
+        }
+      }
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    // after a timeout, loads may still be in flight: wait for them (bounded)
+    for (int st = 0; st < NST; ++st)
+      if ((inflight >> st) & 1u) mbar_wait(&bar[st], (phase >> st) & 1u);
+    bulk_wait_all();
+    if (timeout) atomicOr(&a.stats->status, EP_DEV_WAIT_TIMEOUT);
+  }
+  if (__any_sync(kFull, overflow) && lane == 0) atomicOr(&a.stats->status, EP_DEV_OUT_CAPACITY);
+}
+
+// ---------------------------------------------------------------------------
 // Combine: the reverse of the dispatch.  One warp per token at a time
 // (grid-stride): lanes 0..K-1 fetch the token's dispatch rows and gate
 // weights, lane K its shared-slot row; the warp walks the hidden dimension in
@@ -450,13 +602,13 @@ k_clear_replicas(const int32_t* __restrict__ rep_nexp, const int32_t* __restrict
 }  // namespace
 
 cudaError_t set_copy_attributes(int max_smem) {
-  (void)max_smem;  // the copy kernels use no dynamic shared memory
-  return cudaSuccess;
+  // only the bulk-copy dispatch variant uses dynamic shared memory
+  return allow_max_dynamic_smem(k_permute_bulk<kBulkStages, kBulkAhead>, max_smem);
 }
 
 cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden, void* out,
                             int64_t cap_rows, int rank_begin, int rank_end, int64_t token_begin,
-                            int64_t token_end, int num_sms, cudaStream_t st) {
+                            int64_t token_end, int num_sms, int bulk, cudaStream_t st) {
   PermuteArgs a;
   a.hidden = static_cast<const uint4*>(hidden);
   a.out = static_cast<uint4*>(out);
@@ -476,6 +628,20 @@ cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden
   // measured 6.0 (8), 6.1-6.2 (12) and 6.1 (16) TB/s on the qwen layer;
   // a short token range needs no more than one warp per token
   const int64_t warps = (a.N - a.n0);
+  if (bulk) {
+    const size_t smem = (size_t)kBulkStages * a.row16 * 16;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, k_permute_bulk<kBulkStages, kBulkAhead>, 32, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm > 0 && a.K + 1 <= 32) {
+      const int64_t cap = (int64_t)num_sms * per_sm;
+      const int64_t grid = warps < cap ? warps : cap;
+      k_permute_bulk<kBulkStages, kBulkAhead><<<(unsigned)grid, 32, smem, st>>>(a);
+      return cudaPeekAtLastError();
+    }
+    // rows too large for the ring: the register-staged form below
+  }
   const int64_t blocks = (warps + kPermuteThreads / 32 - 1) / (kPermuteThreads / 32);
   const int64_t grid = blocks < (int64_t)num_sms * 12 ? blocks : (int64_t)num_sms * 12;
   const bool w32 = a.row16 % 2 == 0 && (reinterpret_cast<uintptr_t>(hidden) & 31u) == 0 &&

@@ -126,7 +126,7 @@ cudaError_t launch_balance(const Dims& d, const LayerBuf& L, const Scratch& s,
                            const int32_t* ids, cudaStream_t st);
 cudaError_t launch_dispatch(const Dims& d, const LayerBuf& L, const void* hidden, void* out,
                             int64_t cap_rows, int rank_begin, int rank_end, int64_t token_begin,
-                            int64_t token_end, int num_sms, cudaStream_t st);
+                            int64_t token_end, int num_sms, int bulk, cudaStream_t st);
 cudaError_t launch_combine(const Dims& d, const LayerBuf& L, const void* x, const float* w, void* out,
                            int out_f32, int num_sms, cudaStream_t st);
 cudaError_t launch_stage(const Dims& d, const LayerBuf& L, const void* native_w, void* slots,

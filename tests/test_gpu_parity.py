@@ -216,6 +216,41 @@ def test_plan_deterministic():
         np.testing.assert_array_equal(a[k], b[k])
 
 
+def test_results_do_not_depend_on_the_copy_grids(monkeypatch):
+    # the same layer through plans whose copy kernels run on grids sized for 3
+    # and for 1000 SMs instead of the device's: every output bitwise equal
+    w = get_config("dsv3").replace(T=1000)
+    ids = topk_ids(get_config("dsv3"))[:, :1000].copy()
+    Wn = 3 * 7168 * 2
+    g = torch.Generator(device="cuda")
+    g.manual_seed(31)
+    hidden = torch.randn((w.N, w.hidden), generator=g, device="cuda").to(torch.bfloat16)
+    native = torch.randn((w.E, Wn), generator=g, device="cuda").to(torch.bfloat16)
+    grads = (torch.randn((w.R, w.S, Wn), generator=g, device="cuda") * 1e-2).to(torch.bfloat16)
+    gates = torch.rand((w.R, w.T, w.K), generator=g, device="cuda")
+    outs = []
+    for sms in (None, "3", "1000"):
+        if sms is None:
+            monkeypatch.delenv("EP_GRID_SMS", raising=False)
+        else:
+            monkeypatch.setenv("EP_GRID_SMS", sms)
+        plan = gpu_plan(w, ids, expert_weight_elems=Wn)
+        disp = plan.dispatch_layout(0, hidden)
+        slots = torch.zeros((w.R, w.S, Wn), dtype=torch.bfloat16, device="cuda")
+        plan.stage_replicas(0, native, slots)
+        gr = grads.clone()
+        nat = torch.ones((w.E, Wn), dtype=torch.float32, device="cuda")
+        plan.reduce_replica_grads(0, gr, nat)
+        y = plan.combine(0, disp, gates, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        outs.append([t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+                     for t in (disp, slots, gr, nat, y)] + [plan.view(0)["dst_row"].clone()])
+    monkeypatch.delenv("EP_GRID_SMS", raising=False)
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert torch.equal(a, b)
+
+
 def test_plan_invariants_on_gpu_output():
     w = get_config("qwen")
     ids = topk_ids(w)
@@ -466,6 +501,53 @@ def test_dispatch_token_ranges_match_oracle(shared):
     plan.dispatch_tokens(0, hidden, out, 7, 7)  # empty range: nothing
     torch.cuda.synchronize()
     np.testing.assert_array_equal(out.view(torch.int16).cpu().numpy(), want)
+    assert plan.read_layer_stats(0)["status"] == 0
+
+
+@pytest.mark.parametrize("shared,hidden_dim", [(False, 256), (True, 264), (True, 7168)])
+def test_bulk_copy_dispatch_variant_matches_oracle(monkeypatch, shared, hidden_dim):
+    # the bulk-copy (TMA) variant of the dispatch, chosen at plan creation:
+    # the whole layout, destination-rank windows and source-token ranges give
+    # the oracle's bytes
+    monkeypatch.setenv("EP_DISPATCH_IMPL", "bulk")
+    w = get_config("tiny").replace(T=777, shared_expert=shared, hidden=hidden_dim)
+    ids = topk_ids(get_config("tiny"))[:, :777].copy()
+    plan = gpu_plan(w, ids)
+    monkeypatch.delenv("EP_DISPATCH_IMPL")
+    hidden = _hidden(w, 11)
+    o = oracle_plan(w, ids)
+    want = oracle.permute(o, hidden.view(torch.int16).cpu().numpy())
+    out = plan.dispatch_layout(0, hidden)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.view(torch.int16).cpu().numpy()[: o.rows], want)
+    rb = o.inst_off[np.arange(w.R + 1) * o.G]
+    for b, e in [(0, 1), (1, 4)]:
+        n = int(rb[e] - rb[b])
+        part = plan.dispatch_layout(0, hidden, rank_begin=b, rank_end=e, out_rows=max(n, 1))
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(part.view(torch.int16).cpu().numpy()[:n], want[rb[b]:rb[e]])
+    out2 = torch.zeros_like(out)
+    for lo, hi in [(0, 5), (5, 1500), (1500, w.N)]:
+        plan.dispatch_tokens(0, hidden, out2, lo, hi)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out2.view(torch.int16).cpu().numpy()[: o.rows], want)
+    assert plan.read_layer_stats(0)["status"] == 0
+
+
+def test_bulk_copy_dispatch_variant_full_qwen_round_trip(monkeypatch):
+    monkeypatch.setenv("EP_DISPATCH_IMPL", "bulk")
+    w = get_config("qwen")
+    ids = topk_ids(w)
+    plan = gpu_plan(w, ids)
+    monkeypatch.delenv("EP_DISPATCH_IMPL")
+    hidden = _hidden(w, 12)
+    out = torch.full((w.A, w.hidden), -1.0, dtype=torch.bfloat16, device="cuda")
+    plan.dispatch_layout(0, hidden, out=out)
+    torch.cuda.synchronize()
+    o = oracle_plan(w, ids)
+    dst = o.dst_row.reshape(w.N, w.K)
+    for k in range(w.K):  # the oracle's rows hold the tokens
+        assert _rows_hold_tokens(out, 0, o.rows, np.ascontiguousarray(dst[:, k]), hidden) == w.N
     assert plan.read_layer_stats(0)["status"] == 0
 
 

@@ -167,6 +167,8 @@ def _workload(args):
     if w.layers > 1:
         w = w.replace(layers=1)
     over = {}
+    if getattr(args, "rerouting", "local") == "sampled":
+        over["sampled_rerouting"] = True
     if args.tokens_per_rank is not None:
         over["T"] = args.tokens_per_rank
     if args.ffn is not None:
@@ -705,6 +707,8 @@ def main():
     ap.add_argument("--tokens-per-rank", type=int, default=None,
                     help="override T (small cases for profiler captures)")
     ap.add_argument("--ffn", type=int, default=None, help="override the expert FFN width")
+    ap.add_argument("--rerouting", default="local", choices=["local", "sampled"],
+                    help="rerouting mode of the timed workload (local-first, or per-token sampling)")
     ap.add_argument("--dispatch-impl", default="regs", choices=["regs", "bulk"],
                     help="dispatch kernel: register-staged (default) or the bulk-copy (TMA) "
                          "variant, for comparing the two")

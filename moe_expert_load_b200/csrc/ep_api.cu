@@ -28,10 +28,10 @@ struct Layout {
       shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, inst_count, stats;
   size_t layer_bytes;
   // scratch (absolute)
-  size_t sub_cnt, blk_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_rel, inst_rel, slack, wf, sbase,
+  size_t sub_cnt, blk_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_base, inst_rel, slack, wf, sbase,
       shared_tot, asg_rank, smp_cum, smp_inst, smp_key, smp_sub, smp_blk, smp_row0, rank_rows,
       prev_base,
-      acc_load, acc_tot, acc_misc, smp_tot;
+      acc_load, acc_misc, smp_tot;
   size_t acc_end;  // end of the accumulators zeroed before a plan's first balance call
   size_t scratch_bytes;
   size_t total;
@@ -124,7 +124,7 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.seg_ptr = s.take(i4 * (size_t)d.E * (d.R + 1));
   L.seg_ord = s.take(i4 * (size_t)d.E * 3 * d.R);
   L.seg_rank = s.take(i4 * (size_t)d.E * 3 * d.R);
-  L.seg_rel = s.take(i4 * (size_t)d.E * 3 * d.R);
+  L.seg_base = s.take(i4 * (size_t)d.E * 3 * d.R);
   L.inst_rel = s.take(i4 * (size_t)d.R * d.G);
   L.slack = s.take(i4 * d.R);
   L.wf = s.take(i4 * 2);
@@ -143,7 +143,6 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.prev_base = s.take(i4 * (d.R + 1));
   // contiguous: zeroed together once, before the plan's first balance call
   L.acc_load = s.take(i4 * (size_t)d.R * d.E);
-  L.acc_tot = s.take(i4 * d.E);
   L.acc_misc = s.take(i4 * 4);
   L.smp_tot = s.take(i4 * (size_t)d.R * nk);
   L.acc_end = s.off;
@@ -207,7 +206,7 @@ ep::Scratch scratch(const ep_plan* p) {
   s.seg_ptr = at(p, l.seg_ptr);
   s.seg_ord = at(p, l.seg_ord);
   s.seg_rank = at(p, l.seg_rank);
-  s.seg_rel = at(p, l.seg_rel);
+  s.seg_base = at(p, l.seg_base);
   s.inst_rel = at(p, l.inst_rel);
   s.slack = at(p, l.slack);
   s.wf = at(p, l.wf);
@@ -215,7 +214,6 @@ ep::Scratch scratch(const ep_plan* p) {
   s.shared_tot = at(p, l.shared_tot);
   s.asg_rank = p->d.sh ? reinterpret_cast<uint8_t*>(p->ws + l.asg_rank) : nullptr;
   s.acc_load = at(p, l.acc_load);
-  s.acc_tot = at(p, l.acc_tot);
   s.acc_misc = at(p, l.acc_misc);
   const bool smp = p->d.sampled;
   s.smp_tot = smp ? at(p, l.smp_tot) : nullptr;

@@ -68,7 +68,8 @@ struct Scratch {
   int32_t* seg_ptr;   // [E][R+1] first segment of each source rank, per expert
   int32_t* seg_ord;   // [E][3R] first ordinal of the segment
   int32_t* seg_rank;  // [E][3R] destination rank
-  int32_t* seg_rel;   // [E][3R] first row, relative to the destination rank's block
+  int32_t* seg_base;  // [E][3R] first row minus first ordinal: absolute without a shared
+                      // expert, relative to the destination rank's block with one
   int32_t* inst_rel;  // [R*G] first row of an instance inside its rank's block
   int32_t* slack;     // [R] Waterfill slack
   int32_t* wf;        // [2] Waterfill H, B
@@ -76,10 +77,10 @@ struct Scratch {
   int32_t* shared_tot;  // [R] shared-slot rows per destination rank
   uint8_t* asg_rank;    // [R][T][K] destination rank of each assignment (shared expert only)
   // Accumulators that are zero whenever no balance call is running: the
-  // histogram adds into them, the solve and the rerouting copy them out to the
-  // layer and zero them again, and the arrival ticket resets itself.
+  // histogram adds into the load matrix, the rerouting copies it out to the
+  // layer and zeroes it again, the solve moves the status bits, and the
+  // arrival ticket resets itself.
   int32_t* acc_load;    // [R][E]
-  int32_t* acc_tot;     // [E]
   int32_t* acc_misc;    // [0] status bits of the histogram, [1] arrival ticket
   // Sampled rerouting mode only.  An instance key is kappa = e + rep_eptr[e] + j
   // for the j-th instance of expert e in instance order (E + R*S keys at most).

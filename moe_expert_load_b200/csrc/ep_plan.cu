@@ -57,9 +57,9 @@ constexpr int kAsgBatch = 8;   // ids per lane per pass in k_assign
 // shared-memory histogram with shared atomic adds; the warp writes its row of
 // counts and the block writes the sum of its rows (the two levels of bases of
 // the stable ordinals, used by k_assign).  The block then adds its sum to the
-// load-matrix and expert-total accumulators with integer atomics
-// (order-independent, so the result is deterministic); they are zero on entry
-// and the solve and the rerouting move them into the layer.  The first kernel
+// load-matrix accumulator with integer atomics (order-independent, so the
+// result is deterministic); it is zero on entry, the solve sums its columns
+// into the expert totals and the rerouting moves it into the layer.  The first kernel
 // of the plan: a plain launch, so the ids are complete when it starts.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, 6)
@@ -112,10 +112,7 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
 #pragma unroll
   for (int u = 0; u < kExpPerThread; ++u) {
     const int e = threadIdx.x + u * blockDim.x;
-    if (e < E && csum[u]) {
-      atomicAdd(&s.acc_load[r * E + e], csum[u]);
-      atomicAdd(&s.acc_tot[e], csum[u]);
-    }
+    if (e < E && csum[u]) atomicAdd(&s.acc_load[r * E + e], csum[u]);
   }
 }
 
@@ -169,8 +166,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   int32_t* Tot = sm;              // [E]
   int32_t* Qn_all = sm + d.E;     // [J][E]
   int32_t* cnt_e = Qn_all + d.J * d.E;  // [E+1]
-  int32_t* s_eptr = cnt_e + d.E + 1;    // [E+1] replica-list offsets
-  int32_t* s_rel = s_eptr + d.E + 1;    // [R*G] rank-relative first rows
+  int32_t* s_rel = cnt_e + d.E + 1;     // [R*G] rank-relative first rows
   __shared__ int32_t s_W0[kMaxR];
   __shared__ int32_t s_Wf[kMaxR];
   __shared__ int32_t s_se[kMaxR * kMaxS];
@@ -178,6 +174,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   __shared__ int32_t s_cmax[kMaxJ], s_crep[kMaxJ], s_cstop[kMaxJ];
   __shared__ int32_t s_best, s_A, s_iter_cap_hit;
   __shared__ int32_t s_base[kMaxR + 1];
+  __shared__ int32_t s_wsum[kMaxJ];
 
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -188,12 +185,29 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
 
   pdl_trigger();
   pdl_wait();
-  for (int e = tid; e < E; e += nthr) {
-    const int v = s.acc_tot[e];
-    Tot[e] = v;
-    L.expert_total[e] = v;
-    s.acc_tot[e] = 0;  // zero again for the next call
+  // expert totals: the load matrix's columns summed over source ranks (the
+  // histogram adds only into the load matrix: one total per expert would
+  // take an atomic from every block of the grid)
+  for (int e = tid; e < E; e += nthr) Tot[e] = 0;
+  __syncthreads();
+  {
+    const int n = R * E;  // consecutive threads read consecutive experts of one rank
+    int x = tid;
+    for (; x + 3 * nthr < n; x += 4 * nthr) {
+      int v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = s.acc_load[x + u * nthr];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v[u]) atomicAdd(&Tot[(x + u * nthr) % E], v[u]);
+    }
+    for (; x < n; x += nthr) {
+      const int v = s.acc_load[x];
+      if (v) atomicAdd(&Tot[x % E], v);
+    }
   }
+  __syncthreads();
+  for (int e = tid; e < E; e += nthr) L.expert_total[e] = Tot[e];
   if (tid == 0) {
     s_iter_cap_hit = 0;
     L.stats->status = s.acc_misc[0];  // the first status bits of this call
@@ -472,42 +486,47 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     }
     for (int q = tid; q < R; q += nthr) s.slack[q] = (int)max(H - (int64_t)s_Wf[q], (int64_t)0);
   }
-  // replica lists grouped by expert (CSR), instance order inside an expert
-  if (warp == 0) {
-    int carry = 0, ncarry = 0;
-    for (int e0 = 0; e0 <= E; e0 += 32) {
-      const int e = e0 + lane;
-      const int v = e < E ? cnt_e[e] : 0;
-      const int f = v > 0 ? 1 : 0;
-      int incl = v, fincl = f;
+  // replica lists grouped by expert (CSR): the offsets rep_eptr and the list
+  // of replicated experts come from one block-wide exclusive scan of
+  // (replicas of e) | (e has replicas) << 16 — both sums stay below 2^16 —
+  // and k_reroute writes each expert's slots into its part of the list
+  {
+    constexpr int kIPT = (kMaxE + 1 + kMaxJ * 32 - 1) / (kMaxJ * 32);
+    int vals[kIPT], local = 0;
+#pragma unroll
+    for (int u = 0; u < kIPT; ++u) {
+      const int e = tid * kIPT + u;
+      const int c = e < E ? cnt_e[e] : 0;
+      vals[u] = c | (c > 0 ? 1 << 16 : 0);
+      local += vals[u];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = lane < nthr / 32 ? s_wsum[lane] : 0;
+      int wi = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, incl, o);
-        const int z = __shfl_up_sync(kFull, fincl, o);
-        if (lane >= o) { incl += y; fincl += z; }
+        const int y = __shfl_up_sync(kFull, wi, o);
+        if (lane >= o) wi += y;
       }
-      if (e <= E) {
-        L.rep_eptr[e] = carry + incl - v;
-        s_eptr[e] = carry + incl - v;
-      }
-      if (e < E && f) L.rep_experts[ncarry + fincl - 1] = e;
-      carry += __shfl_sync(kFull, incl, 31);
-      ncarry += __shfl_sync(kFull, fincl, 31);
+      if (lane < nthr / 32) s_wsum[lane] = wi - v;
     }
-    if (lane == 0) L.rep_nexp[0] = ncarry;
-    // each filled slot's place in its expert's list: the list's start plus
-    // the earlier slots of that expert (32 slots at a time, in slot order)
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) cnt_e[e] = s_eptr[e];
-    __syncwarp();
-    for (int i0 = 0; i0 < R * S; i0 += 32) {
-      const int i = i0 + lane;
-      const int e = i < R * S ? s_se[i] : -1;
-      const unsigned peers = __match_any_sync(kFull, e);
-      if (e >= 0) L.rep_list[cnt_e[e] + __popc(peers & lanemask_lt())] = i;
-      __syncwarp();
-      if (e >= 0 && lane == __ffs(peers) - 1) cnt_e[e] += __popc(peers);
-      __syncwarp();
+    __syncthreads();
+    int run = s_wsum[warp] + incl - local;
+#pragma unroll
+    for (int u = 0; u < kIPT; ++u) {
+      const int e = tid * kIPT + u;
+      if (e <= E) L.rep_eptr[e] = run & 0xffff;
+      if (e < E && (vals[u] & 0xffff)) L.rep_experts[run >> 16] = e;
+      if (e == E) L.rep_nexp[0] = run >> 16;
+      run += vals[u];
     }
   }
 }
@@ -528,10 +547,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   __shared__ int32_t s_iloc[kWarpsPerBlock][kMaxR];   // instance j: local take
   __shared__ int32_t s_jof[kWarpsPerBlock][kMaxR];    // rank -> instance j or -1
   __shared__ int32_t s_igi[kWarpsPerBlock][kMaxR];    // instance j: global instance index
+  __shared__ int32_t s_rb[kMaxR + 1];                 // first row of each rank (no shared expert)
   pdl_trigger();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * kWarpsPerBlock + warp;
+  if (!d.sh && !d.sampled)
+    for (int q = threadIdx.x; q <= d.R; q += blockDim.x) s_rb[q] = L.rank_base[q];
+  __syncthreads();
   if (e >= d.E) return;
   const int R = d.R, E = d.E, G = d.G, S = d.S;
   int32_t* irank = s_irank[warp];
@@ -566,6 +589,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   // after the replicas on ranks below h.  Every slot's entries are loaded in
   // one round, independent of each other.
   int nrep = 0, np = 0;
+  int32_t* rlist = L.rep_list + L.rep_eptr[e];  // e's part of the replica list
   for (int i0 = 0; i0 < R * S; i0 += 32) {
     const int i = i0 + lane;
     const int q = i / S, col = d.Gmax + (i - (i / S) * S);
@@ -578,6 +602,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
     }
     const unsigned m = __ballot_sync(kFull, hit);
     if (hit) {
+      rlist[nrep + __popc(m & lanemask_lt())] = i;  // slot order = instance order
       const int j = nrep + __popc(m & lanemask_lt()) + (q > h ? 1 : 0);
       irank[j] = q;
       irel[j] = rel;
@@ -714,7 +739,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   // pass 2: write the segments
   int32_t* sord = s.seg_ord + (int64_t)e * 3 * R;
   int32_t* srank = s.seg_rank + (int64_t)e * 3 * R;
-  int32_t* srel = s.seg_rel + (int64_t)e * 3 * R;
+  int32_t* sbase = s.seg_base + (int64_t)e * 3 * R;
+  // a segment's rows start at its destination rank's first row (without a
+  // shared expert; with one, k_fixup adds it later) plus its offset there
+  const bool absolute = !d.sh;
 #pragma unroll
   for (int k = 0; k < kRW; ++k) {
     const int r = lane + 32 * k;
@@ -726,7 +754,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
       const int before = min(max(PD[k] - ipq[j], 0), iq[j]);  // remote rows of earlier sources
       sord[w] = 0;
       srank[w] = r;
-      srel[w] = irel[j] + before;
+      sbase[w] = (absolute ? s_rb[r] : 0) + irel[j] + before;
       ++w;
     }
     if (Dr[k] > 0) {
@@ -735,9 +763,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
         if (iq[j] <= 0) continue;
         const int lo = max(PD[k], ipq[j]);
         const int c = irank[j];
-        sord[w] = locr[k] + (lo - PD[k]);
+        const int ord = locr[k] + (lo - PD[k]);
+        sord[w] = ord;
         srank[w] = c;
-        srel[w] = irel[j] + (c < r ? iloc[j] : 0) + (lo - ipq[j]);
+        sbase[w] = (absolute ? s_rb[c] : 0) + irel[j] + (c < r ? iloc[j] : 0) + (lo - ipq[j]) - ord;
         ++w;
       }
     }
@@ -885,6 +914,81 @@ __host__ __device__ __forceinline__ int seg_capacity(const Dims& d) {
 }
 
 template <int PASS>
+struct AssignCtx {
+  const int4* sge;       // [E+1] per-expert first-segment records (slot E: dummy)
+  int32_t* run;          // [E+1] the warp's running ordinals
+  const int32_t* sg_ord;
+  const int32_t* sg_base;
+  const int32_t* sg_rank;
+  int32_t* drow;         // dst_row of the source rank
+  uint8_t* grank;        // destination-rank bytes of the source rank (PASS 1)
+  uint8_t* dr;           // the sub-chunk's destination ranks in shared memory (PASS 1)
+  int a0, E, lane;
+  unsigned lt;           // lanes below this one
+};
+
+// One round: assignment idx (of the source rank) with id vv; `in` is false
+// for lanes past the sub-chunk's end.
+template <int PASS, bool FULL>
+__device__ __forceinline__ void assign_one(const AssignCtx<PASS>& c, int vv, int idx, bool in,
+                                           bool& inconsistent) {
+  const bool valid = vv >= 0 && vv < c.E && (FULL || in);
+  const int e = valid ? vv : c.E;
+  const int4 g = c.sge[e];
+  const unsigned peers = __match_any_sync(kFull, e);
+  const int o = c.run[e] + __popc(peers & c.lt);
+  __syncwarp();
+  if (c.lane == __ffs(peers) - 1) c.run[e] = o + __popc(peers);  // the leader's o is the count
+  __syncwarp();
+  const int n = g.y & 0xffff;
+  int b = g.z, q = g.y >> 16;
+  if (o >= g.w) {  // a later segment: the last one starting at or before o
+    int si = g.x + n - 1;
+    while (si > g.x && c.sg_ord[si] > o) --si;
+    b = c.sg_base[si];
+    if (PASS > 0) q = c.sg_rank[si];
+  }
+  const bool ok = valid && n > 0;
+  inconsistent |= valid && n == 0;
+  if (FULL || in) {
+    c.drow[idx] = ok ? b + o : -1;
+    if (PASS > 0) {
+      const uint8_t rank = ok ? (uint8_t)q : (uint8_t)kNoRank;
+      c.dr[idx - c.a0] = rank;
+      c.grank[idx] = rank;
+    }
+  }
+}
+
+// The rounds of one warp's sub-chunk [a0, a1) of the source rank's
+// assignments; v holds the first batch of ids (fetched before the wait).
+template <int PASS, bool FULL>
+__device__ __forceinline__ void assign_rounds(const AssignCtx<PASS>& c, const int32_t* __restrict__ src,
+                                              int a0, int a1, int (&v)[kAsgBatch],
+                                              bool& inconsistent) {
+  for (int a = a0; a < a1; a += kAsgBatch * 32) {
+    if (a != a0) {
+#pragma unroll
+      for (int u = 0; u < kAsgBatch; ++u) {
+        const int idx = a + u * 32 + c.lane;
+        v[u] = (FULL || idx < a1) ? __ldg(src + idx) : -1;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kAsgBatch; ++u) {
+      if (FULL) {
+        if (a + u * 32 >= a1) break;  // K * 64 is a multiple of 32 but maybe not of 256
+        assign_one<PASS, true>(c, v[u], a + u * 32 + c.lane, true, inconsistent);
+      } else {
+        if (a + u * 32 >= a1) break;
+        const int idx = a + u * 32 + c.lane;
+        assign_one<PASS, false>(c, v[u], idx, idx < a1, inconsistent);
+      }
+    }
+  }
+}
+
+template <int PASS>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   extern __shared__ __align__(16) int32_t sm[];
@@ -902,14 +1006,16 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   const int segcap = seg_capacity(d);
   // per expert: {first segment, segment count | first segment's rank << 16,
   // first segment's row - ordinal, second segment's first ordinal (or INT_MAX)}
-  int4* sge = reinterpret_cast<int4*>(sm);              // [E]
-  int32_t* sg_ord = sm + 4 * E;                         // [segcap] first ordinal
+  // slot E of the record table and of the running counts is a dummy that
+  // dropped ids (and lanes past the end of the sub-chunk) share
+  int4* sge = reinterpret_cast<int4*>(sm);              // [E+1]
+  int32_t* sg_ord = sm + 4 * (E + 1);                   // [segcap] first ordinal
   int32_t* sg_base = sg_ord + segcap;                   // [segcap] row - ordinal
   int32_t* sg_rank = sg_base + segcap;                  // [segcap] destination rank
   int32_t* base0 = sg_rank + (PASS > 0 ? segcap : 0);   // [E]
-  const int per_warp = E + (PASS > 0 ? R + (kPlanSubT * K + 3) / 4 : 0);
-  int32_t* run = base0 + E + warp * per_warp;           // [E] running ordinals
-  int32_t* wrun = run + E;                              // [R] running shared ordinals
+  const int per_warp = E + 1 + (PASS > 0 ? R + (kPlanSubT * K + 3) / 4 : 0);
+  int32_t* run = base0 + E + warp * per_warp;           // [E+1] running ordinals
+  int32_t* wrun = run + E + 1;                          // [R] running shared ordinals
   uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);   // [kPlanSubT*K] destination ranks
 
   // The first batch of ids is an input no kernel of the plan writes: fetch it
@@ -962,7 +1068,7 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
         int4 g = make_int4(off, 0, 0, INT_MAX);
         for (int j = 0; j < cnt[u] && off + j < segcap; ++j) {
           const int ord = s.seg_ord[gb + j], rank = s.seg_rank[gb + j];
-          const int base = (PASS == 0 ? L.rank_base[rank] : 0) + s.seg_rel[gb + j] - ord;
+          const int base = s.seg_base[gb + j];
           sg_ord[off + j] = ord;
           sg_base[off + j] = base;
           if (PASS > 0) sg_rank[off + j] = rank;
@@ -977,6 +1083,7 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
         off += cnt[u];
       }
     }
+    if (tid == 0) sge[E] = make_int4(0, 1, 0, INT_MAX);
   }
   // exclusive base of the block's first sub-chunk
   for (int e = tid; e < E; e += nthr) base0[e] = 0;
@@ -1019,55 +1126,21 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     for (int w = 0; w < warp; ++w) acc += cnt_r[(int64_t)(sub0 + w) * E + e];
     run[e] = acc;
   }
+  if (lane == 0) run[E] = 0;
   __syncwarp();
 
+  // Main loop, 32 assignments per round: the stable ordinal of an assignment
+  // is its expert's running count plus its rank inside the round's match.any
+  // group (the group's leader advances the count).  The expert's segment record
+  // is fetched before the match, and a full sub-chunk (every one but a rank's
+  // last) runs without per-element bounds checks.
   bool inconsistent = false;
-  for (int a = a0; a < a1; a += kAsgBatch * 32) {
-    if (a != a0) {
-#pragma unroll
-      for (int u = 0; u < kAsgBatch; ++u) {
-        const int idx = a + u * 32 + lane;
-        v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kAsgBatch; ++u) {
-      if (a + u * 32 >= a1) break;
-      const int idx = a + u * 32 + lane;
-      const int e = (v[u] >= 0 && v[u] < E) ? v[u] : -1;
-      const unsigned peers = __match_any_sync(kFull, e);
-      const int rk = __popc(peers & lanemask_lt());
-      const int o = e >= 0 ? run[e] + rk : 0;
-      __syncwarp();
-      if (e >= 0 && lane == __ffs(peers) - 1) run[e] = o + __popc(peers);  // leader: rk = 0
-      __syncwarp();
-      if (idx < a1) {
-        int row = -1, rank = kNoRank;
-        if (e >= 0) {
-          const int4 g = sge[e];
-          const int n = g.y & 0xffff;
-          if (n > 0) {
-            int b = g.z, q = g.y >> 16;
-            if (o >= g.w) {  // a later segment: the last one starting at or before o
-              int si = g.x + n - 1;
-              while (si > g.x && sg_ord[si] > o) --si;
-              b = sg_base[si];
-              if (PASS > 0) q = sg_rank[si];
-            }
-            row = b + o;
-            if (PASS > 0) rank = q;
-          } else {
-            inconsistent = true;
-          }
-        }
-        L.dst_row[rbase + idx] = row;
-        if (PASS > 0) {
-          dr[idx - a0] = (uint8_t)rank;
-          s.asg_rank[rbase + idx] = (uint8_t)rank;
-        }
-      }
-    }
-  }
+  AssignCtx<PASS> c{sge, run, sg_ord, sg_base, sg_rank, L.dst_row + rbase,
+                    PASS > 0 ? s.asg_rank + rbase : nullptr, dr, a0, E, lane, lanemask_lt()};
+  if (a1 - a0 == kPlanSubT * K)
+    assign_rounds<PASS, true>(c, ids + rbase, a0, a1, v, inconsistent);
+  else
+    assign_rounds<PASS, false>(c, ids + rbase, a0, a1, v, inconsistent);
   if (__any_sync(kFull, inconsistent) && lane == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
   if (PASS > 0) waterfill_subchunk(d, L, s, r, sub, t0, t1, dr, wrun, s_slack, s_W, lane);
 }
@@ -1160,13 +1233,14 @@ k_sample(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   }
 }
 
-// k_sample_layout: one CTA.  Per key, the exclusive prefix of the draws over
-// source ranks (rows of earlier sources come first inside an instance) and
-// the key's total, which is its instance's row count; the accumulator is
-// zeroed for the next call.  Then the rank-relative first row of every
-// instance, each rank's routed rows, the dispatch layout (without a shared
-// expert; with one, k_shared_scan lays the ranks out) and the first row of
-// every (source rank, key), absolute or rank-relative.
+// k_sample_layout: one CTA, a thread per key (consecutive keys read
+// consecutive words of each source rank's row, eight rows in flight).  Pass 1:
+// the key's draws summed over source ranks, which is its instance's row
+// count.  Then the rank-relative first row of every instance, each rank's
+// routed rows and the dispatch layout (without a shared expert; with one,
+// k_shared_scan lays the ranks out).  Pass 2: the first row of every (source
+// rank, key) — the instance's first row plus the draws of earlier sources —
+// absolute or rank-relative; the accumulator is zeroed for the next call.
 constexpr int kLayoutThreads = 1024;
 
 __global__ void __launch_bounds__(kLayoutThreads) k_sample_layout(Dims d, LayerBuf L, Scratch s) {
@@ -1186,15 +1260,17 @@ __global__ void __launch_bounds__(kLayoutThreads) k_sample_layout(Dims d, LayerB
   for (int i = tid; i < RG; i += kLayoutThreads) s_icnt[i] = 0;
   __syncthreads();
   const int nk = s_nk;
-  for (int k = tid; k < nk; k += kLayoutThreads) {
-    int run = 0;
-    for (int r = 0; r < R; ++r) {
-      const int v = s.smp_tot[r * NK + k];
-      s.smp_tot[r * NK + k] = 0;  // zero again for the next call
-      s.smp_row0[r * NK + k] = run;
-      run += v;
+  for (int k = tid; k < nk; k += kLayoutThreads) {  // consecutive keys: coalesced rows
+    int sum = 0, r = 0;
+    for (; r + 8 <= R; r += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = s.smp_tot[(r + u) * NK + k];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += v[u];
     }
-    s_kcnt[k] = run;
+    for (; r < R; ++r) sum += s.smp_tot[r * NK + k];
+    s_kcnt[k] = sum;
     s_kinst[k] = s.smp_inst[k];
   }
   __syncthreads();
@@ -1244,12 +1320,28 @@ __global__ void __launch_bounds__(kLayoutThreads) k_sample_layout(Dims d, LayerB
     }
     for (int q = tid; q <= R; q += kLayoutThreads) L.rank_base[q] = s_base[q];
   }
-  for (int x = tid; x < R * nk; x += kLayoutThreads) {
-    const int r = x / nk, k = x - (x / nk) * nk;
+  for (int k = tid; k < nk; k += kLayoutThreads) {
     const int i = s_kinst[k];
-    if (i < 0 || i >= RG) continue;
-    const int first = d.sh ? s_rel[i] : s_base[i / G] + s_rel[i];
-    s.smp_row0[r * NK + k] += first;
+    if (i < 0 || i >= RG) continue;  // every key has an instance; guard the tables anyway
+    int run = d.sh ? s_rel[i] : s_base[i / G] + s_rel[i];
+    int r = 0;
+    for (; r + 8 <= R; r += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = s.smp_tot[(r + u) * NK + k];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        s.smp_row0[(r + u) * NK + k] = run;
+        s.smp_tot[(r + u) * NK + k] = 0;  // zero again for the next call
+        run += v[u];
+      }
+    }
+    for (; r < R; ++r) {
+      const int v = s.smp_tot[r * NK + k];
+      s.smp_row0[r * NK + k] = run;
+      s.smp_tot[r * NK + k] = 0;
+      run += v;
+    }
   }
 }
 
@@ -1628,14 +1720,14 @@ size_t wf_layer_smem(const Dims& d) {
   return sizeof(int32_t) * (size_t)kWarpsPerBlock * (d.R + (kPlanSubT * d.K + 3) / 4);
 }
 size_t solve_smem(const Dims& d) {
-  return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + 2 * ((size_t)d.E + 1) + (size_t)d.R * d.G);
+  return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + ((size_t)d.E + 1) + (size_t)d.R * d.G);
 }
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
   const size_t segcap = (size_t)seg_capacity(d);
-  const size_t per_warp = d.E + (pass > 0 ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
-  return sizeof(int32_t) *
-         (4 * (size_t)d.E + segcap * (pass > 0 ? 3 : 2) + d.E + (size_t)kWarpsPerBlock * per_warp);
+  const size_t per_warp = d.E + 1 + (pass > 0 ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
+  return sizeof(int32_t) * (4 * ((size_t)d.E + 1) + segcap * (pass > 0 ? 3 : 2) + d.E +
+                            (size_t)kWarpsPerBlock * per_warp);
 }
 
 // Launch with programmatic stream serialisation: the kernel may begin while

@@ -79,6 +79,13 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     line = bench.run_reference(Args())
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["cores"] == 1
+    # the step as run: its wall time, not the whole-layer estimate the value uses
+    cb = line["cpu_baseline"]
+    assert line["ms_per_step"] == cb["ms_per_step_measured"]
+    assert line["steps"] * line["ms_per_step"] <= 1e3 * line["wall_s"] + 1.0
+    assert cb["oracle_plan_ms"] > 0 and cb["host_cpu_count"] >= 1 and "cpu_model" in cb
+    # both arms describe the workload with the same config
+    assert line["config"] == bench._config(bench._workload(Args()), 2)
 
 
 def test_traffic_record_hash_ignores_comments(tmp_path):

@@ -30,6 +30,23 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
+// Lanes of the warp whose key equals this lane's, for keys below 2^nbits
+// (nbits <= 12): the intersection of one ballot per key bit.  Measured on
+// B200 in the sampled-mode assignment (qwen / dsv3 plan 93 -> 87 / 148 -> 141
+// us against match.any); in the local-first assignment and the Waterfill pass
+// it was slower (stress 168 -> 194 us) and match.any stays there.
+__device__ __forceinline__ unsigned match_bits(int key, int nbits) {
+  unsigned m = kFull;
+#pragma unroll
+  for (int b = 0; b < 12; ++b) {
+    if (b >= nbits) break;  // warp-uniform
+    const bool bit = (key >> b) & 1;
+    const unsigned bal = __ballot_sync(kFull, bit);
+    m &= bit ? bal : ~bal;
+  }
+  return m;
+}
+
 // SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the state is advanced by the
 // golden-gamma increment and finished with the variant-13 mixer.
 __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
@@ -79,7 +96,7 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
     const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
     const int32_t* src = ids + (int64_t)r * d.T * K;
     const int a1 = t1 * K;
-    for (int a = t0 * K; a < a1; a += kBatch * 32) {  // one pass for K <= 16
+    for (int a = t0 * K; a < a1; a += kBatch * 32) {  // one pass for K <= 8, two for K <= 16
       int v[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
@@ -160,7 +177,7 @@ __device__ __forceinline__ int warp_argmax_rank(const unsigned (&v)[RW], const b
 // number of 32-rank words) and keeps their load, slot table and flags in
 // registers; native quotas live in shared memory.
 // ---------------------------------------------------------------------------
-template <int SMAX, int RW>
+template <int SMAX, int RW, bool PACK>
 __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scratch s) {
   extern __shared__ int32_t sm[];
   int32_t* Tot = sm;              // [E]
@@ -183,27 +200,34 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   // division here rather than one per greedy step
   const int eb = E / R, er = E - (E / R) * R;
 
-  pdl_trigger();
+  // wait first: the rerouting, launched at this trigger, may then read the
+  // histogram's load matrix before waiting for the solve
   pdl_wait();
+  pdl_trigger();
   // expert totals: the load matrix's columns summed over source ranks (the
   // histogram adds only into the load matrix: one total per expert would
   // take an atomic from every block of the grid)
   for (int e = tid; e < E; e += nthr) Tot[e] = 0;
   __syncthreads();
   {
-    const int n = R * E;  // consecutive threads read consecutive experts of one rank
-    int x = tid;
-    for (; x + 3 * nthr < n; x += 4 * nthr) {
-      int v[4];
+    // thread (slice, e) sums ranks slice, slice + nslice, ... of expert e:
+    // consecutive threads read consecutive experts of a rank, eight loads in
+    // flight, one shared-memory add per thread at the end
+    const int nslice = E < nthr ? nthr / E : 1;
+    for (int t = tid; t < nslice * E; t += nthr) {
+      const int e = t % E, sl = t / E;
+      int acc = 0;
+      for (int r = sl; r < R; r += 8 * nslice) {  // eight loads issued together
+        int v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = s.acc_load[x + u * nthr];
+        for (int u = 0; u < 8; ++u) {
+          const int q = r + u * nslice;
+          v[u] = q < R ? s.acc_load[q * E + e] : 0;
+        }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (v[u]) atomicAdd(&Tot[(x + u * nthr) % E], v[u]);
-    }
-    for (; x < n; x += nthr) {
-      const int v = s.acc_load[x];
-      if (v) atomicAdd(&Tot[x % E], v);
+        for (int u = 0; u < 8; ++u) acc += v[u];
+      }
+      if (acc) atomicAdd(&Tot[e], acc);
     }
   }
   __syncthreads();
@@ -259,8 +283,10 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     }
     __syncwarp();
     const int iter_cap = d.iter_limit > 0 ? d.iter_limit : 4 * (R * S + R + E) + 64;
-    // every key value is a load, a slack or a quota: at most C <= 1.08 A
-    const bool pack = A < (1 << 24);
+    // every key value is a load, a slack or a quota, at most C <= 1.08 A: below
+    // 2^25 whenever R*T*K < 2^24 (the host's choice of PACK), so value and
+    // index travel in one 32-bit redux key
+    constexpr bool pack = PACK;
     for (int it = 0;; ++it) {
       if (it >= iter_cap) { stop = EP_STOP_ITER_CAP; break; }
       unsigned wv[RW];
@@ -547,16 +573,25 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   __shared__ int32_t s_iloc[kWarpsPerBlock][kMaxR];   // instance j: local take
   __shared__ int32_t s_jof[kWarpsPerBlock][kMaxR];    // rank -> instance j or -1
   __shared__ int32_t s_igi[kWarpsPerBlock][kMaxR];    // instance j: global instance index
-  __shared__ int32_t s_rb[kMaxR + 1];                 // first row of each rank (no shared expert)
+  __shared__ int32_t s_rbw[kWarpsPerBlock][kMaxR + 1];  // first row of each rank, per warp
   pdl_trigger();
-  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * kWarpsPerBlock + warp;
-  if (!d.sh && !d.sampled)
-    for (int q = threadIdx.x; q <= d.R; q += blockDim.x) s_rb[q] = L.rank_base[q];
-  __syncthreads();
-  if (e >= d.E) return;
   const int R = d.R, E = d.E, G = d.G, S = d.S;
+  // the load column of e: the histogram had completed before the solve
+  // triggered this launch, so it is read before waiting for the solve (which
+  // reads the load matrix too: it is copied out and zeroed only after the wait)
+  int lcol[kRW];
+#pragma unroll
+  for (int k = 0; k < kRW; ++k) {
+    const int r = lane + 32 * k;
+    lcol[k] = (e < E && r < R) ? s.acc_load[r * E + e] : 0;
+  }
+  pdl_wait();
+  if (e >= d.E) return;
+  int32_t* s_rb = s_rbw[warp];
+  if (!d.sh && !d.sampled)  // issued now, read once the segments are written
+    for (int q = lane; q <= d.R; q += 32) s_rb[q] = L.rank_base[q];
   int32_t* irank = s_irank[warp];
   int32_t* irel = s_irel[warp];
   int32_t* iq = s_iq[warp];
@@ -565,18 +600,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   int32_t* jof = s_jof[warp];
   int32_t* igi = s_igi[warp];
 
-  // the load column of e: independent of the instance lookups below, so its
-  // loads are issued first
-  int lcol[kRW];
 #pragma unroll
   for (int k = 0; k < kRW; ++k) {
     const int r = lane + 32 * k;
     if (r < R) {
-      lcol[k] = s.acc_load[r * E + e];
       L.load[r * E + e] = lcol[k];
       s.acc_load[r * E + e] = 0;  // zero again for the next call
-    } else {
-      lcol[k] = 0;
     }
   }
   const int h = home_of(e, E, R);
@@ -916,7 +945,6 @@ __host__ __device__ __forceinline__ int seg_capacity(const Dims& d) {
 template <int PASS>
 struct AssignCtx {
   const int4* sge;       // [E+1] per-expert first-segment records (slot E: dummy)
-  int32_t* run;          // [E+1] the warp's running ordinals
   const int32_t* sg_ord;
   const int32_t* sg_base;
   const int32_t* sg_rank;
@@ -927,19 +955,11 @@ struct AssignCtx {
   unsigned lt;           // lanes below this one
 };
 
-// One round: assignment idx (of the source rank) with id vv; `in` is false
-// for lanes past the sub-chunk's end.
-template <int PASS, bool FULL>
-__device__ __forceinline__ void assign_one(const AssignCtx<PASS>& c, int vv, int idx, bool in,
-                                           bool& inconsistent) {
-  const bool valid = vv >= 0 && vv < c.E && (FULL || in);
-  const int e = valid ? vv : c.E;
-  const int4 g = c.sge[e];
-  const unsigned peers = __match_any_sync(kFull, e);
-  const int o = c.run[e] + __popc(peers & c.lt);
-  __syncwarp();
-  if (c.lane == __ffs(peers) - 1) c.run[e] = o + __popc(peers);  // the leader's o is the count
-  __syncwarp();
+// The row (and destination rank) of ordinal o of an expert whose first-segment
+// record is g; ok is false for a dropped id or an expert without segments.
+template <int PASS>
+__device__ __forceinline__ void assign_finish(const AssignCtx<PASS>& c, const int4& g, int o,
+                                              bool valid, int idx, bool in, bool& inconsistent) {
   const int n = g.y & 0xffff;
   int b = g.z, q = g.y >> 16;
   if (o >= g.w) {  // a later segment: the last one starting at or before o
@@ -950,7 +970,7 @@ __device__ __forceinline__ void assign_one(const AssignCtx<PASS>& c, int vv, int
   }
   const bool ok = valid && n > 0;
   inconsistent |= valid && n == 0;
-  if (FULL || in) {
+  if (in) {
     c.drow[idx] = ok ? b + o : -1;
     if (PASS > 0) {
       const uint8_t rank = ok ? (uint8_t)q : (uint8_t)kNoRank;
@@ -960,30 +980,41 @@ __device__ __forceinline__ void assign_one(const AssignCtx<PASS>& c, int vv, int
   }
 }
 
+// One round: assignment idx (of the source rank) with id vv; `in` is false
+// for lanes past the sub-chunk's end.
+template <int PASS>
+__device__ __forceinline__ void assign_one(const AssignCtx<PASS>& c, int32_t* run, int vv, int idx,
+                                           bool in, bool& inconsistent) {
+  const bool valid = in && vv >= 0 && vv < c.E;
+  const int e = valid ? vv : c.E;
+  const int4 g = c.sge[e];
+  const unsigned peers = __match_any_sync(kFull, e);
+  const int o = run[e] + __popc(peers & c.lt);
+  __syncwarp();
+  if (c.lane == __ffs(peers) - 1) run[e] = o + __popc(peers);  // the leader's o is the count
+  __syncwarp();
+  assign_finish<PASS>(c, g, o, valid, idx, in, inconsistent);
+}
+
 // The rounds of one warp's sub-chunk [a0, a1) of the source rank's
 // assignments; v holds the first batch of ids (fetched before the wait).
-template <int PASS, bool FULL>
+template <int PASS>
 __device__ __forceinline__ void assign_rounds(const AssignCtx<PASS>& c, const int32_t* __restrict__ src,
-                                              int a0, int a1, int (&v)[kAsgBatch],
-                                              bool& inconsistent) {
+                                              int32_t* run, int a0, int a1,
+                                              int (&v)[kAsgBatch], bool& inconsistent) {
   for (int a = a0; a < a1; a += kAsgBatch * 32) {
     if (a != a0) {
 #pragma unroll
       for (int u = 0; u < kAsgBatch; ++u) {
         const int idx = a + u * 32 + c.lane;
-        v[u] = (FULL || idx < a1) ? __ldg(src + idx) : -1;
+        v[u] = idx < a1 ? __ldg(src + idx) : -1;
       }
     }
 #pragma unroll
     for (int u = 0; u < kAsgBatch; ++u) {
-      if (FULL) {
-        if (a + u * 32 >= a1) break;  // K * 64 is a multiple of 32 but maybe not of 256
-        assign_one<PASS, true>(c, v[u], a + u * 32 + c.lane, true, inconsistent);
-      } else {
-        if (a + u * 32 >= a1) break;
-        const int idx = a + u * 32 + c.lane;
-        assign_one<PASS, false>(c, v[u], idx, idx < a1, inconsistent);
-      }
+      if (a + u * 32 >= a1) break;  // warp-uniform
+      const int idx = a + u * 32 + c.lane;
+      assign_one<PASS>(c, run, v[u], idx, idx < a1, inconsistent);
     }
   }
 }
@@ -1131,16 +1162,12 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
 
   // Main loop, 32 assignments per round: the stable ordinal of an assignment
   // is its expert's running count plus its rank inside the round's match.any
-  // group (the group's leader advances the count).  The expert's segment record
-  // is fetched before the match, and a full sub-chunk (every one but a rank's
-  // last) runs without per-element bounds checks.
+  // group (the group's leader advances the count).  The expert's segment record is fetched before the match, off the
+  // chain; dropped ids and lanes past the end share the dummy slot E.
   bool inconsistent = false;
-  AssignCtx<PASS> c{sge, run, sg_ord, sg_base, sg_rank, L.dst_row + rbase,
+  AssignCtx<PASS> c{sge, sg_ord, sg_base, sg_rank, L.dst_row + rbase,
                     PASS > 0 ? s.asg_rank + rbase : nullptr, dr, a0, E, lane, lanemask_lt()};
-  if (a1 - a0 == kPlanSubT * K)
-    assign_rounds<PASS, true>(c, ids + rbase, a0, a1, v, inconsistent);
-  else
-    assign_rounds<PASS, false>(c, ids + rbase, a0, a1, v, inconsistent);
+  assign_rounds<PASS>(c, ids + rbase, run, a0, a1, v, inconsistent);
   if (__any_sync(kFull, inconsistent) && lane == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
   if (PASS > 0) waterfill_subchunk(d, L, s, r, sub, t0, t1, dr, wrun, s_slack, s_W, lane);
 }
@@ -1419,7 +1446,7 @@ k_sample_assign(Dims d, LayerBuf L, Scratch s) {
       if (a + u * 32 >= a1) break;
       const int idx = a + u * 32 + lane;
       const int key = v[u] < nk ? v[u] : -1;
-      const unsigned peers = __match_any_sync(kFull, key);
+      const unsigned peers = match_bits(key >= 0 ? key : nk, 32 - __clz(nk));
       const int rk = __popc(peers & lanemask_lt());
       const int o = key >= 0 ? run[key] + rk : 0;
       __syncwarp();
@@ -1725,7 +1752,7 @@ size_t solve_smem(const Dims& d) {
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
   const size_t segcap = (size_t)seg_capacity(d);
-  const size_t per_warp = d.E + 1 + (pass > 0 ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
+  const size_t per_warp = (size_t)d.E + 1 + (pass > 0 ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
   return sizeof(int32_t) * (4 * ((size_t)d.E + 1) + segcap * (pass > 0 ? 3 : 2) + d.E +
                             (size_t)kWarpsPerBlock * per_warp);
 }
@@ -1752,13 +1779,18 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
 
 // Allow every kernel the device's opt-in shared-memory maximum once, so that
 // plans of any shape can coexist (each launch still requests only its own size).
+template <int SMAX, bool PACK>
+cudaError_t allow_solve_pack(int max_smem) {
+  cudaError_t e;
+  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 1, PACK>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 2, PACK>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 3, PACK>, max_smem)) != cudaSuccess) return e;
+  return allow_max_dynamic_smem(k_solve<SMAX, 4, PACK>, max_smem);
+}
 template <int SMAX>
 cudaError_t allow_solve(int max_smem) {
-  cudaError_t e;
-  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 1>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 2>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 3>, max_smem)) != cudaSuccess) return e;
-  return allow_max_dynamic_smem(k_solve<SMAX, 4>, max_smem);
+  cudaError_t e = allow_solve_pack<SMAX, true>(max_smem);
+  return e != cudaSuccess ? e : allow_solve_pack<SMAX, false>(max_smem);
 }
 
 cudaError_t set_plan_attributes(int max_smem) {
@@ -1782,10 +1814,16 @@ cudaError_t launch_solve_rw(const Dims& d, const LayerBuf& L, const Scratch& s, 
   const size_t ss = solve_smem(d);
   const unsigned nt = kMaxJ * 32;
   const int rw = (d.R + 31) / 32;
-  if (rw <= 1) return launch_pdl(k_solve<SMAX, 1>, 1, nt, ss, st, d, L, s);
-  if (rw == 2) return launch_pdl(k_solve<SMAX, 2>, 1, nt, ss, st, d, L, s);
-  if (rw == 3) return launch_pdl(k_solve<SMAX, 3>, 1, nt, ss, st, d, L, s);
-  return launch_pdl(k_solve<SMAX, 4>, 1, nt, ss, st, d, L, s);
+  if ((int64_t)d.R * d.T * d.K < ((int64_t)1 << 24)) {
+    if (rw <= 1) return launch_pdl(k_solve<SMAX, 1, true>, 1, nt, ss, st, d, L, s);
+    if (rw == 2) return launch_pdl(k_solve<SMAX, 2, true>, 1, nt, ss, st, d, L, s);
+    if (rw == 3) return launch_pdl(k_solve<SMAX, 3, true>, 1, nt, ss, st, d, L, s);
+    return launch_pdl(k_solve<SMAX, 4, true>, 1, nt, ss, st, d, L, s);
+  }
+  if (rw <= 1) return launch_pdl(k_solve<SMAX, 1, false>, 1, nt, ss, st, d, L, s);
+  if (rw == 2) return launch_pdl(k_solve<SMAX, 2, false>, 1, nt, ss, st, d, L, s);
+  if (rw == 3) return launch_pdl(k_solve<SMAX, 3, false>, 1, nt, ss, st, d, L, s);
+  return launch_pdl(k_solve<SMAX, 4, false>, 1, nt, ss, st, d, L, s);
 }
 
 cudaError_t launch_solve(const Dims& d, const LayerBuf& L, const Scratch& s, cudaStream_t st) {

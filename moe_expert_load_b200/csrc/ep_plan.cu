@@ -1061,9 +1061,49 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
   }
   pdl_trigger();
+
+  // Before waiting: the histogram's counts.  The histogram finished before the
+  // solve passed its own wait and triggered the rerouting, whose trigger
+  // launched this grid, so its block and sub-chunk counts are complete here.
+  // The exclusive base of the block's first sub-chunk (earlier blocks of this
+  // rank), then each warp's running counts (plus the block's earlier warps).
+  for (int e = tid; e < E; e += nthr) base0[e] = 0;
+  __syncthreads();
+  const int32_t* cnt_r = s.sub_cnt + (int64_t)r * d.nsub * E;
+  {
+    const int32_t* blk_r = s.blk_cnt + (int64_t)r * nbpr * E;
+    const int n = (sub0 / kWarpsPerBlock) * E;
+    for (int i = tid; i < n; i += nthr * 8) {
+      int c[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int ii = i + u * nthr;
+        c[u] = ii < n ? blk_r[ii] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int ii = i + u * nthr;
+        if (c[u]) atomicAdd(&base0[ii % E], c[u]);
+      }
+    }
+  }
+  __syncthreads();
+  if (active) {
+    for (int e = lane; e < E; e += 32) {
+      int c[kWarpsPerBlock];  // the block's earlier warps' counts, loaded together
+#pragma unroll
+      for (int w = 0; w < kWarpsPerBlock; ++w)
+        c[w] = w < warp ? cnt_r[(int64_t)(sub0 + w) * E + e] : 0;
+      int acc = base0[e];
+#pragma unroll
+      for (int w = 0; w < kWarpsPerBlock; ++w) acc += c[w];
+      run[e] = acc;
+    }
+    if (lane == 0) run[E] = 0;
+  }
   pdl_wait();
 
-  // rank r's segment table
+  // rank r's segment table (the rerouting's output)
   {
     const int per = (E + nthr - 1) / nthr;
     const int eb = tid * per;
@@ -1116,49 +1156,17 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     }
     if (tid == 0) sge[E] = make_int4(0, 1, 0, INT_MAX);
   }
-  // exclusive base of the block's first sub-chunk
-  for (int e = tid; e < E; e += nthr) base0[e] = 0;
-  for (int q = tid; q < R; q += nthr) {
-    if (PASS > 0) {
+  if (PASS > 0)
+    for (int q = tid; q < R; q += nthr) {
       s_slack[q] = s.slack[q];
       s_W[q] = L.W[q];
-
     }
-  }
   __syncthreads();
-  const bool overflow = s_total > segcap;
-  if (overflow) {
+  if (s_total > segcap) {
     if (tid == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
     return;
   }
-  const int32_t* cnt_r = s.sub_cnt + (int64_t)r * d.nsub * E;
-  {
-    // blocks of this rank before this one: their per-block counts
-    const int32_t* blk_r = s.blk_cnt + (int64_t)r * nbpr * E;
-    const int n = (sub0 / kWarpsPerBlock) * E;
-    for (int i = tid; i < n; i += nthr * 8) {
-      int c[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int ii = i + u * nthr;
-        c[u] = ii < n ? blk_r[ii] : 0;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int ii = i + u * nthr;
-        if (c[u]) atomicAdd(&base0[ii % E], c[u]);
-      }
-    }
-  }
-  __syncthreads();
   if (!active) return;
-  for (int e = lane; e < E; e += 32) {
-    int acc = base0[e];
-    for (int w = 0; w < warp; ++w) acc += cnt_r[(int64_t)(sub0 + w) * E + e];
-    run[e] = acc;
-  }
-  if (lane == 0) run[E] = 0;
-  __syncwarp();
 
   // Main loop, 32 assignments per round: the stable ordinal of an assignment
   // is its expert's running count plus its rank inside the round's match.any
@@ -1200,6 +1208,18 @@ k_sample(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   int32_t* s_tot = s_eptr + E + 1;     // [E]
   int32_t* hists = s_tot + E;          // [warps][NK]
   int32_t* hist = hists + warp * NK;
+  // the first batch of ids is an input no kernel of the plan writes: fetch it
+  // before waiting
+  const bool active = sub < d.nsub;
+  const int t0 = active ? sub * kPlanSubT : 0, t1 = active ? min(d.T, t0 + kPlanSubT) : 0;
+  const int64_t rbase = (int64_t)r * d.T * K;
+  const int a1 = t1 * K;
+  int v[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) {
+    const int idx = t0 * K + u * 32 + lane;
+    v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
+  }
   pdl_trigger();
   pdl_wait();
   for (int e = tid; e <= E; e += nthr) s_eptr[e] = L.rep_eptr[e];
@@ -1209,16 +1229,14 @@ k_sample(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   for (int i = tid; i < nk; i += nthr) s_cum[i] = s.smp_cum[i];
   for (int i = lane; i < nk; i += 32) hist[i] = 0;
   __syncthreads();
-  if (sub < d.nsub) {
-    const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
-    const int64_t rbase = (int64_t)r * d.T * K;
-    const int a1 = t1 * K;
+  if (active) {
     for (int a = t0 * K; a < a1; a += kBatch * 32) {
-      int v[kBatch];
+      if (a != t0 * K) {
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int idx = a + u * 32 + lane;
-        v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
+        for (int u = 0; u < kBatch; ++u) {
+          const int idx = a + u * 32 + lane;
+          v[u] = idx < a1 ? __ldg(ids + rbase + idx) : -1;
+        }
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
@@ -1281,8 +1299,10 @@ __global__ void __launch_bounds__(kLayoutThreads) k_sample_layout(Dims d, LayerB
   int32_t* s_kinst = s_kcnt + NK;  // [NK] instance of the key
   int32_t* s_icnt = s_kinst + NK;  // [R*G] rows per instance
   int32_t* s_rel = s_icnt + RG;    // [R*G] rank-relative first row
-  pdl_trigger();
+  // wait first: the assignment pass, launched at this trigger, may then read
+  // the sampling pass's draws before waiting for this layout
   pdl_wait();
+  pdl_trigger();
   if (tid == 0) s_nk = E + L.rep_eptr[E];
   for (int i = tid; i < RG; i += kLayoutThreads) s_icnt[i] = 0;
   __syncthreads();
@@ -1401,36 +1421,51 @@ k_sample_assign(Dims d, LayerBuf L, Scratch s) {
   int32_t* wrun = run + NK;                    // [R] running shared ordinals (SH)
   uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);  // [kPlanSubT*K] ranks (SH)
   pdl_trigger();
-  pdl_wait();
+  // Before waiting: the draws (the sampling pass had completed before the
+  // layout passed its own wait and launched this grid) — the exclusive base
+  // of the block's first sub-chunk and each warp's running counts.
   if (tid == 0) s_nk = E + L.rep_eptr[E];
   __syncthreads();
   const int nk = s_nk;
-  for (int k = tid; k < nk; k += nthr) {
-    s_row0[k] = s.smp_row0[r * NK + k];
-    if (SH) s_krank[k] = s.smp_inst[k] / G;
-    base0[k] = 0;
+  {
+    const int32_t* blk_r = s.smp_blk + (int64_t)r * nbpr * NK;
+    const int nb = sub0 / kWarpsPerBlock;
+    for (int k = tid; k < nk; k += nthr) {
+      int acc = 0;
+      for (int b0 = 0; b0 < nb; b0 += 8) {  // eight loads in flight
+        int c[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) c[u] = b0 + u < nb ? blk_r[(int64_t)(b0 + u) * NK + k] : 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc += c[u];
+      }
+      base0[k] = acc;
+      if (SH) s_krank[k] = s.smp_inst[k] / G;
+    }
   }
+  __syncthreads();
+  const int32_t* cnt_r = s.smp_sub + (int64_t)r * d.nsub * NK;
+  if (active) {
+    for (int k = lane; k < nk; k += 32) {
+      int c[kWarpsPerBlock];
+#pragma unroll
+      for (int w = 0; w < kWarpsPerBlock; ++w)
+        c[w] = w < warp ? cnt_r[(int64_t)(sub0 + w) * NK + k] : 0;
+      int acc = base0[k];
+#pragma unroll
+      for (int w = 0; w < kWarpsPerBlock; ++w) acc += c[w];
+      run[k] = acc;
+    }
+  }
+  pdl_wait();
+  for (int k = tid; k < nk; k += nthr) s_row0[k] = s.smp_row0[r * NK + k];
   if (SH)
     for (int q = tid; q < R; q += nthr) {
       s_slack[q] = s.slack[q];
       s_W[q] = L.W[q];
     }
   __syncthreads();
-  {
-    const int32_t* blk_r = s.smp_blk + (int64_t)r * nbpr * NK;
-    const int nb = sub0 / kWarpsPerBlock;
-    for (int b = 0; b < nb; ++b)
-      for (int k = tid; k < nk; k += nthr) base0[k] += blk_r[(int64_t)b * NK + k];
-  }
-  __syncthreads();
   if (!active) return;
-  const int32_t* cnt_r = s.smp_sub + (int64_t)r * d.nsub * NK;
-  for (int k = lane; k < nk; k += 32) {
-    int acc = base0[k];
-    for (int w = 0; w < warp; ++w) acc += cnt_r[(int64_t)(sub0 + w) * NK + k];
-    run[k] = acc;
-  }
-  __syncwarp();
   const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
   const int a0 = t0 * K, a1 = t1 * K;
   const int64_t rbase = (int64_t)r * d.T * K;
@@ -1559,8 +1594,10 @@ __global__ void __launch_bounds__(kScanThreads) k_shared_scan(Dims d, LayerBuf L
   __shared__ int32_t s_carry;
   __shared__ int32_t s_last;
   __shared__ int32_t s_base[kMaxR + 1];
-  pdl_trigger();
+  // wait first: the fix-up, launched at this trigger, may then read the
+  // assignment pass's rows and rank bytes before waiting for this scan
   pdl_wait();
+  pdl_trigger();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int R = d.R, G = d.G;
   const int c = blockIdx.x;
@@ -1653,13 +1690,7 @@ __global__ void __launch_bounds__(kFixThreads) k_fixup(Dims d, LayerBuf L, Scrat
   __shared__ int32_t s_rb[kMaxR + 1];
   __shared__ int32_t s_sb[kMaxR];
   pdl_trigger();
-  pdl_wait();
   const int R = d.R;
-  for (int q = threadIdx.x; q <= R; q += blockDim.x) {
-    s_rb[q] = L.rank_base[q];
-    if (q < R) s_sb[q] = s.sbase[q];
-  }
-  __syncthreads();
   const int64_t A = (int64_t)R * d.T * d.K;
   const int N = R * d.T;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -1668,9 +1699,23 @@ __global__ void __launch_bounds__(kFixThreads) k_fixup(Dims d, LayerBuf L, Scrat
   const int64_t A4 = A / 4;
   int4* row4 = reinterpret_cast<int4*>(L.dst_row);
   const uint32_t* rk4 = reinterpret_cast<const uint32_t*>(s.asg_rank);
+  // the first rows and rank bytes: the assignment pass that wrote them had
+  // completed before the shared scan passed its wait and launched this grid
+  int4 v0 = make_int4(0, 0, 0, 0);
+  uint32_t q0w = 0;
+  if (i0 < A4) {
+    v0 = row4[i0];
+    q0w = rk4[i0];
+  }
+  pdl_wait();
+  for (int q = threadIdx.x; q <= R; q += blockDim.x) {
+    s_rb[q] = L.rank_base[q];
+    if (q < R) s_sb[q] = s.sbase[q];
+  }
+  __syncthreads();
   for (int64_t i = i0; i < A4; i += stride) {
-    int4 v = row4[i];
-    const uint32_t q = rk4[i];
+    int4 v = i == i0 ? v0 : row4[i];
+    const uint32_t q = i == i0 ? q0w : rk4[i];
     const int q0 = q & 0xffu, q1 = (q >> 8) & 0xffu, q2 = (q >> 16) & 0xffu, q3 = q >> 24;
     // a rank byte is a rank below R, or kNoRank for a dropped assignment;
     // anything else leaves the row alone

@@ -63,7 +63,8 @@ enum {
 /* Device status bits (ep_layer_stats.status). */
 #define EP_DEV_BAD_ID 1        /* a top-k id outside [0, E): not counted, its row is -1 */
 #define EP_DEV_ITER_CAP 2      /* a cap candidate hit the solver's iteration bound */
-#define EP_DEV_WAIT_TIMEOUT 4  /* reserved for bounded waits (no current kernel waits) */
+#define EP_DEV_WAIT_TIMEOUT 4  /* a bounded wait ran out (the bulk-copy dispatch variant's
+                                  mbarrier waits; the default kernels never wait) */
 #define EP_DEV_OUT_CAPACITY 8  /* a dispatch row fell outside the caller's output buffer */
 #define EP_DEV_INCONSISTENT 16 /* an assignment found no rerouting segment (internal check) */
 

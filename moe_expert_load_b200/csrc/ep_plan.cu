@@ -10,11 +10,14 @@
 // the Waterfill page §"Waterfill" (waterline H, slack, per-token draw).
 // Everything is integer arithmetic; all orders are fixed, so results are
 // bit-identical run to run and independent of the grid size.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <limits.h>
 #include <stdint.h>
 
 #include "ep_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace ep {
 namespace {
@@ -177,22 +180,27 @@ __device__ __forceinline__ int warp_argmax_rank(const unsigned (&v)[RW], const b
 // number of 32-rank words) and keeps their load, slot table and flags in
 // registers; native quotas live in shared memory.
 // ---------------------------------------------------------------------------
+constexpr int kSolveWarps = 4;                     // cap candidates per CTA: one per SM partition
+constexpr int kSolveThreads = kSolveWarps * 32;
+
 template <int SMAX, int RW, bool PACK>
-__global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scratch s) {
+__global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, Scratch s) {
   extern __shared__ int32_t sm[];
   int32_t* Tot = sm;              // [E]
-  int32_t* Qn_all = sm + d.E;     // [J][E]
-  int32_t* cnt_e = Qn_all + d.J * d.E;  // [E+1]
+  int32_t* Qn_all = sm + d.E;     // [kSolveWarps][E]: this CTA's candidates' native quotas
+  int32_t* cnt_e = Qn_all + kSolveWarps * d.E;  // [E+1]
   int32_t* s_rel = cnt_e + d.E + 1;     // [R*G] rank-relative first rows
   __shared__ int32_t s_W0[kMaxR];
   __shared__ int32_t s_Wf[kMaxR];
   __shared__ int32_t s_se[kMaxR * kMaxS];
   __shared__ int32_t s_sq[kMaxR * kMaxS];
   __shared__ int32_t s_cmax[kMaxJ], s_crep[kMaxJ], s_cstop[kMaxJ];
-  __shared__ int32_t s_best, s_A, s_iter_cap_hit;
+  __shared__ int32_t s_best, s_A, s_iter_cap_hit, s_tight, s_any_cap;
   __shared__ int32_t s_base[kMaxR + 1];
   __shared__ int32_t s_wsum[kMaxJ];
 
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = (int)cluster.block_rank(), ncta = (int)cluster.num_blocks();
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int R = d.R, E = d.E, S = d.S, m = d.m;
@@ -206,44 +214,53 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   pdl_trigger();
   // expert totals: the load matrix's columns summed over source ranks (the
   // histogram adds only into the load matrix: one total per expert would
-  // take an atomic from every block of the grid)
-  for (int e = tid; e < E; e += nthr) Tot[e] = 0;
+  // take an atomic from every block of the grid).  CTA c of the cluster sums
+  // experts [c*E/n, (c+1)*E/n) — thread (slice, e) sums ranks slice,
+  // slice + nslice, ... of expert e, sixteen loads in flight — and every CTA
+  // then reads the other CTAs' totals from their shared memory.
+  const int e_lo = crank * E / ncta, e_hi = (crank + 1) * E / ncta, ne = e_hi - e_lo;
+  for (int e = e_lo + tid; e < e_hi; e += nthr) Tot[e] = 0;
+  if (tid == 0) s_iter_cap_hit = 0;
   __syncthreads();
-  {
-    // thread (slice, e) sums ranks slice, slice + nslice, ... of expert e:
-    // consecutive threads read consecutive experts of a rank, eight loads in
-    // flight, one shared-memory add per thread at the end
-    const int nslice = E < nthr ? nthr / E : 1;
-    for (int t = tid; t < nslice * E; t += nthr) {
-      const int e = t % E, sl = t / E;
+  if (ne > 0) {
+    const int nslice = ne < nthr ? nthr / ne : 1;
+    for (int t = tid; t < nslice * ne; t += nthr) {
+      const int e = e_lo + t % ne, sl = t / ne;
       int acc = 0;
-      for (int r = sl; r < R; r += 8 * nslice) {  // eight loads issued together
-        int v[8];
+      for (int r = sl; r < R; r += 16 * nslice) {
+        int v[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 16; ++u) {
           const int q = r + u * nslice;
           v[u] = q < R ? s.acc_load[q * E + e] : 0;
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc += v[u];
+        for (int u = 0; u < 16; ++u) acc += v[u];
       }
       if (acc) atomicAdd(&Tot[e], acc);
     }
   }
-  __syncthreads();
-  for (int e = tid; e < E; e += nthr) L.expert_total[e] = Tot[e];
-  if (tid == 0) {
-    s_iter_cap_hit = 0;
-    L.stats->status = s.acc_misc[0];  // the first status bits of this call
-    s.acc_misc[0] = 0;
+  cluster.sync();
+  for (int e = tid; e < E; e += nthr) {
+    if (e >= e_lo && e < e_hi) continue;
+    int c = 0;
+    while (e >= (c + 1) * E / ncta) ++c;  // the CTA whose range holds e
+    Tot[e] = *cluster.map_shared_rank(&Tot[e], c);
   }
   __syncthreads();
+  if (crank == 0) {
+    for (int e = tid; e < E; e += nthr) L.expert_total[e] = Tot[e];
+    if (tid == 0) {
+      L.stats->status = s.acc_misc[0];  // the first status bits of this call
+      s.acc_misc[0] = 0;
+    }
+  }
   if (tid < R) {
     const int f = tid * eb + min(tid, er), n = eb + (tid < er ? 1 : 0);
     int w = 0;
     for (int i = 0; i < n; ++i) w += Tot[f + i];
     s_W0[tid] = w;
-    L.W0[tid] = w;
+    if (crank == 0) L.W0[tid] = w;
   }
   __syncthreads();
   if (warp == 0) {
@@ -256,21 +273,21 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
     bm = (int)__reduce_max_sync(kFull, (unsigned)bm);
     if (lane == 0) {
       s_A = a;
-      L.stats->before_max = bm;
+      if (crank == 0) L.stats->before_max = bm;
     }
   }
   __syncthreads();
   const int A = s_A;
 
-  // ---- one greedy run per warp ----
-  const bool solver = warp < d.J;
-  const int j = warp;
+  // ---- one greedy run per warp: candidate j = crank * kSolveWarps + warp ----
+  const int j = crank * kSolveWarps + warp;
+  const bool solver = j < d.J;
   const int64_t den = 200LL * R;
   const int C = (int)(((int64_t)A * (200 + j) + den - 1) / den);
   int Wr[RW], used[RW], se[RW][SMAX], sq[RW][SMAX];
   int replicas = 0, stop = -1, maxW = 0;
   if (solver) {
-    int32_t* Qn = Qn_all + j * E;
+    int32_t* Qn = Qn_all + warp * E;
     for (int e = lane; e < E; e += 32) Qn[e] = Tot[e];
     unsigned stuck = 0, slotlim = 0;
 #pragma unroll
@@ -405,16 +422,29 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       if (stop == EP_STOP_ITER_CAP) atomicOr(&s_iter_cap_hit, 1);
     }
   }
-  __syncthreads();
-  if (warp == 0) {  // smallest (max load, replicas, j)
-    const unsigned k1 = lane < d.J ? (unsigned)s_cmax[lane] : 0xffffffffu;
+  cluster.sync();
+  if (warp == 0) {  // smallest (max load, replicas, j), read from the candidates' CTAs
+    const int owner = lane / kSolveWarps;
+    const bool cand = lane < d.J;
+    const unsigned cmax = cand ? (unsigned)*cluster.map_shared_rank(&s_cmax[lane], owner) : 0u;
+    const unsigned crep = cand ? (unsigned)*cluster.map_shared_rank(&s_crep[lane], owner) : 0u;
+    const int cstop0 = *cluster.map_shared_rank(&s_cstop[0], 0);
+    const bool cap_hit = lane < ncta && *cluster.map_shared_rank(&s_iter_cap_hit, lane);
+    const unsigned k1 = cand ? cmax : 0xffffffffu;
     const unsigned m1 = __reduce_min_sync(kFull, k1);
-    const unsigned k2 = (lane < d.J && k1 == m1) ? (unsigned)s_crep[lane] * 32u + (unsigned)lane
-                                                 : 0xffffffffu;
+    const unsigned k2 = (cand && k1 == m1) ? crep * 32u + (unsigned)lane : 0xffffffffu;
     const unsigned m2 = __reduce_min_sync(kFull, k2);
-    if (lane == 0) s_best = (int)(m2 & 31u);
+    const bool any_cap = __any_sync(kFull, cap_hit);
+    if (lane == 0) {
+      s_best = (int)(m2 & 31u);
+      s_tight = cstop0;
+      s_any_cap = any_cap ? 1 : 0;
+    }
   }
-  __syncthreads();
+  // every remote read above is done before any CTA leaves; only the winner's
+  // CTA lays the plan out
+  cluster.sync();
+  if (crank != s_best / kSolveWarps) return;
   if (solver && j == s_best) {
 #pragma unroll
     for (int k = 0; k < RW; ++k) {
@@ -432,20 +462,20 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
       ep_layer_stats* st = L.stats;
       st->cap_idx = j;
       st->stop_reason = stop;
-      st->tight_stop_reason = s_cstop[0];
+      st->tight_stop_reason = s_tight;
       st->replicas = replicas;
       st->cap = C;
       st->assignments = A;
       st->after_max = maxW;
       st->realized_max = maxW;
-      if (s_iter_cap_hit) atomicOr(&st->status, EP_DEV_ITER_CAP);
+      if (s_any_cap) atomicOr(&st->status, EP_DEV_ITER_CAP);
     }
   }
   __syncthreads();
 
   // ---- emit the winner's instance table ----
   const int G = d.G, Gmax = d.Gmax;
-  const int32_t* Qw = Qn_all + s_best * E;
+  const int32_t* Qw = Qn_all + (s_best % kSolveWarps) * E;
   for (int i = tid; i < R * G; i += nthr) {
     const int q = i / G, col = i - (i / G) * G;
     int ex = -1, qu = 0;
@@ -517,7 +547,7 @@ __global__ void __launch_bounds__(kMaxJ * 32, 1) k_solve(Dims d, LayerBuf L, Scr
   // (replicas of e) | (e has replicas) << 16 — both sums stay below 2^16 —
   // and k_reroute writes each expert's slots into its part of the list
   {
-    constexpr int kIPT = (kMaxE + 1 + kMaxJ * 32 - 1) / (kMaxJ * 32);
+    constexpr int kIPT = (kMaxE + 1 + kSolveThreads - 1) / kSolveThreads;
     int vals[kIPT], local = 0;
 #pragma unroll
     for (int u = 0; u < kIPT; ++u) {
@@ -1792,7 +1822,7 @@ size_t wf_layer_smem(const Dims& d) {
   return sizeof(int32_t) * (size_t)kWarpsPerBlock * (d.R + (kPlanSubT * d.K + 3) / 4);
 }
 size_t solve_smem(const Dims& d) {
-  return sizeof(int32_t) * ((size_t)d.E * (1 + d.J) + ((size_t)d.E + 1) + (size_t)d.R * d.G);
+  return sizeof(int32_t) * ((size_t)d.E * (1 + kSolveWarps) + ((size_t)d.E + 1) + (size_t)d.R * d.G);
 }
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
@@ -1854,21 +1884,44 @@ cudaError_t set_plan_attributes(int max_smem) {
   return allow_max_dynamic_smem(k_sample_assign<1>, max_smem);
 }
 
+// The solve: a cluster of ceil(J / kSolveWarps) CTAs (one cap candidate per
+// warp, at most four per SM), launched as a programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), unsigned ctas, unsigned block, size_t smem,
+                               cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = ctas;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int SMAX>
 cudaError_t launch_solve_rw(const Dims& d, const LayerBuf& L, const Scratch& s, cudaStream_t st) {
   const size_t ss = solve_smem(d);
-  const unsigned nt = kMaxJ * 32;
+  const unsigned nt = kSolveThreads;
+  const unsigned nc = (unsigned)((d.J + kSolveWarps - 1) / kSolveWarps);
   const int rw = (d.R + 31) / 32;
   if ((int64_t)d.R * d.T * d.K < ((int64_t)1 << 24)) {
-    if (rw <= 1) return launch_pdl(k_solve<SMAX, 1, true>, 1, nt, ss, st, d, L, s);
-    if (rw == 2) return launch_pdl(k_solve<SMAX, 2, true>, 1, nt, ss, st, d, L, s);
-    if (rw == 3) return launch_pdl(k_solve<SMAX, 3, true>, 1, nt, ss, st, d, L, s);
-    return launch_pdl(k_solve<SMAX, 4, true>, 1, nt, ss, st, d, L, s);
+    if (rw <= 1) return launch_pdl_cluster(k_solve<SMAX, 1, true>, nc, nt, ss, st, d, L, s);
+    if (rw == 2) return launch_pdl_cluster(k_solve<SMAX, 2, true>, nc, nt, ss, st, d, L, s);
+    if (rw == 3) return launch_pdl_cluster(k_solve<SMAX, 3, true>, nc, nt, ss, st, d, L, s);
+    return launch_pdl_cluster(k_solve<SMAX, 4, true>, nc, nt, ss, st, d, L, s);
   }
-  if (rw <= 1) return launch_pdl(k_solve<SMAX, 1, false>, 1, nt, ss, st, d, L, s);
-  if (rw == 2) return launch_pdl(k_solve<SMAX, 2, false>, 1, nt, ss, st, d, L, s);
-  if (rw == 3) return launch_pdl(k_solve<SMAX, 3, false>, 1, nt, ss, st, d, L, s);
-  return launch_pdl(k_solve<SMAX, 4, false>, 1, nt, ss, st, d, L, s);
+  if (rw <= 1) return launch_pdl_cluster(k_solve<SMAX, 1, false>, nc, nt, ss, st, d, L, s);
+  if (rw == 2) return launch_pdl_cluster(k_solve<SMAX, 2, false>, nc, nt, ss, st, d, L, s);
+  if (rw == 3) return launch_pdl_cluster(k_solve<SMAX, 3, false>, nc, nt, ss, st, d, L, s);
+  return launch_pdl_cluster(k_solve<SMAX, 4, false>, nc, nt, ss, st, d, L, s);
 }
 
 cudaError_t launch_solve(const Dims& d, const LayerBuf& L, const Scratch& s, cudaStream_t st) {

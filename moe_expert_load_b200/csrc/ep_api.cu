@@ -12,6 +12,7 @@
 
 namespace ep {
 cudaError_t set_plan_attributes(int max_smem);
+cudaError_t solve_launch_smem(const Dims& d, int max_smem, int* bytes);
 cudaError_t set_copy_attributes(int max_smem);
 }  // namespace ep
 
@@ -90,6 +91,7 @@ ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
   d->iter_limit = c->solver_iter_limit;
   d->sseed = c->sampling_seed;
   d->nkey = E + R * d->S;  // at most 1024 + 128 * 8 keys: they fit the uint16 key buffer
+  d->solve_smem = 0;       // set at plan creation, from the device's shared-memory limit
   return EP_OK;
 }
 
@@ -288,6 +290,7 @@ ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t works
   if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return EP_ERR_CUDA;
   if (ep::set_plan_attributes(max_smem) != cudaSuccess) return EP_ERR_CUDA;
+  if (ep::solve_launch_smem(d, max_smem, &d.solve_smem) != cudaSuccess) return EP_ERR_CUDA;
   if (ep::set_copy_attributes(max_smem) != cudaSuccess) return EP_ERR_CUDA;
   ep_plan* p = new (std::nothrow) ep_plan;
   if (!p) return EP_ERR_INVALID_ARGUMENT;

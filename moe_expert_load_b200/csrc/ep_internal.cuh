@@ -36,6 +36,7 @@ struct Dims {
   int iter_limit;    // > 0: the solver's iteration bound instead of 4(RS+R+E)+64
   uint64_t sseed;    // seed of the sampled mode's per-assignment draw
   int nkey;          // sampled mode: key space E + R*S (expert-major instance keys)
+  int solve_smem;    // dynamic shared memory of the solve launch (set at plan creation)
 };
 
 // One layer's slot in the plan cache (all device pointers).

@@ -99,17 +99,51 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
     const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
     const int32_t* src = ids + (int64_t)r * d.T * K;
     const int a1 = t1 * K;
-    for (int a = t0 * K; a < a1; a += kBatch * 32) {  // one pass for K <= 8, two for K <= 16
-      int v[kBatch];
+    const int32_t* p = src + t0 * K;
+    const int n = a1 - t0 * K;
+    auto count = [&](int v, bool in) {
+      if (!in) return;
+      if (v < 0 || v >= E) bad = 1;
+      else atomicAdd(&hist[v], 1);  // integer: order-independent
+    };
+    if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+      // 16-byte loads: a lane takes 4 consecutive ids, 4 vectors in flight
+      // (a whole sub-chunk for K <= 8); a vector that would cross the end of
+      // the sub-chunk is read id by id
+      for (int q0 = 0; q0 < n; q0 += 16 * 32) {
+        int4 w[4];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int idx = a + u * 32 + lane;
-        v[u] = idx < a1 ? __ldg(src + idx) : -1;
-        if (idx < a1 && (v[u] < 0 || v[u] >= E)) { bad = 1; v[u] = -1; }
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + 4 * (u * 32 + lane);
+          if (q + 3 < n) {
+            w[u] = __ldg(reinterpret_cast<const int4*>(p + q));
+          } else {
+            w[u].x = q < n ? __ldg(p + q) : -1;
+            w[u].y = q + 1 < n ? __ldg(p + q + 1) : -1;
+            w[u].z = q + 2 < n ? __ldg(p + q + 2) : -1;
+            w[u].w = -1;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + 4 * (u * 32 + lane);
+          count(w[u].x, q < n);
+          count(w[u].y, q + 1 < n);
+          count(w[u].z, q + 2 < n);
+          count(w[u].w, q + 3 < n);
+        }
       }
+    } else {
+      for (int a = t0 * K; a < a1; a += kBatch * 32) {  // one pass for K <= 8, two for K <= 16
+        int v[kBatch];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-        if (v[u] >= 0) atomicAdd(&hist[v[u]], 1);  // integer: order-independent
+        for (int u = 0; u < kBatch; ++u) {
+          const int idx = a + u * 32 + lane;
+          v[u] = idx < a1 ? __ldg(src + idx) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) count(v[u], a + u * 32 + lane < a1);
+      }
     }
     __syncwarp();
     int32_t* out = s.sub_cnt + ((int64_t)r * d.nsub + sub) * E;
@@ -169,7 +203,8 @@ __device__ __forceinline__ int warp_argmax_rank(const unsigned (&v)[RW], const b
 }
 
 // ---------------------------------------------------------------------------
-// a2: quota solve.  One CTA; warp j runs the greedy at cap
+// a2: quota solve.  A thread-block cluster of ceil(J/4) CTAs of 4 warps, one
+// SM each; warp j of the cluster (CTA j/4) runs the greedy at cap
 // C_j = ceil(A (200 + j) / (200 R)).  Greedy step: the most-loaded rank p that is
 // not stuck (smallest index on ties) gives min(max(W_p - C, m), slack_r, Q_e) of
 // its native e — natives tried by quota descending, then expert ascending, only
@@ -966,6 +1001,12 @@ __device__ __forceinline__ void waterfill_subchunk(const Dims& d, const LayerBuf
 // and the sub-chunk's pick counts per destination rank; k_fixup adds the rank
 // bases once the shared columns are laid out.
 // ---------------------------------------------------------------------------
+// The token assignment keeps an assignment's expert (<= E <= 1024, 11 bits)
+// and ordinal in one word when every ordinal of a source rank is below 2^21.
+__host__ __device__ __forceinline__ bool assign_packed(const Dims& d) {
+  return (int64_t)d.T * d.K <= ((int64_t)1 << 21);
+}
+
 __host__ __device__ __forceinline__ int seg_capacity(const Dims& d) {
   // per source rank: at most one local segment per expert, and the remote
   // overlaps of an expert are at most its number of instances
@@ -1010,47 +1051,51 @@ __device__ __forceinline__ void assign_finish(const AssignCtx<PASS>& c, const in
   }
 }
 
-// One round: assignment idx (of the source rank) with id vv; `in` is false
-// for lanes past the sub-chunk's end.
-template <int PASS>
-__device__ __forceinline__ void assign_one(const AssignCtx<PASS>& c, int32_t* run, int vv, int idx,
-                                           bool in, bool& inconsistent) {
-  const bool valid = in && vv >= 0 && vv < c.E;
-  const int e = valid ? vv : c.E;
-  const int4 g = c.sge[e];
-  const unsigned peers = __match_any_sync(kFull, e);
-  const int o = run[e] + __popc(peers & c.lt);
-  __syncwarp();
-  if (c.lane == __ffs(peers) - 1) run[e] = o + __popc(peers);  // the leader's o is the count
-  __syncwarp();
-  assign_finish<PASS>(c, g, o, valid, idx, in, inconsistent);
-}
-
-// The rounds of one warp's sub-chunk [a0, a1) of the source rank's
-// assignments; v holds the first batch of ids (fetched before the wait).
-template <int PASS>
-__device__ __forceinline__ void assign_rounds(const AssignCtx<PASS>& c, const int32_t* __restrict__ src,
-                                              int32_t* run, int a0, int a1,
-                                              int (&v)[kAsgBatch], bool& inconsistent) {
+// The stable ordinals of one warp's sub-chunk [a0, a1) of the source rank's
+// assignments, in rounds of 32: an assignment's ordinal is its expert's
+// running count plus its rank inside the round's match.any group (the group's
+// leader advances the count).  Only the ids and the histogram's counts enter,
+// so this runs before the wait for the rerouting.  so/se receive each
+// assignment's ordinal and expert (E for a dropped id); when every ordinal is
+// below 2^21 (pk) both travel in so as o | e << 21 and se is unused.  v holds
+// the first batch of ids.
+__device__ __forceinline__ void assign_ordinals(const int32_t* __restrict__ src, int32_t* run,
+                                                int a0, int a1, int E, int lane, unsigned lt,
+                                                bool pk, int (&v)[kAsgBatch], int32_t* so,
+                                                uint16_t* se) {
   for (int a = a0; a < a1; a += kAsgBatch * 32) {
     if (a != a0) {
 #pragma unroll
       for (int u = 0; u < kAsgBatch; ++u) {
-        const int idx = a + u * 32 + c.lane;
+        const int idx = a + u * 32 + lane;
         v[u] = idx < a1 ? __ldg(src + idx) : -1;
       }
     }
 #pragma unroll
     for (int u = 0; u < kAsgBatch; ++u) {
       if (a + u * 32 >= a1) break;  // warp-uniform
-      const int idx = a + u * 32 + c.lane;
-      assign_one<PASS>(c, run, v[u], idx, idx < a1, inconsistent);
+      const int idx = a + u * 32 + lane;
+      const bool in = idx < a1;
+      const int e = in && v[u] >= 0 && v[u] < E ? v[u] : E;
+      const unsigned peers = __match_any_sync(kFull, e);
+      const int o = run[e] + __popc(peers & lt);
+      __syncwarp();
+      if (lane == __ffs(peers) - 1) run[e] = o + __popc(peers);  // the leader's o is the count
+      __syncwarp();
+      if (in) {
+        if (pk) {
+          so[idx - a0] = (int32_t)((unsigned)o | ((unsigned)e << 21));
+        } else {
+          so[idx - a0] = o;
+          se[idx - a0] = (uint16_t)e;
+        }
+      }
     }
   }
 }
 
 template <int PASS>
-__global__ void __launch_bounds__(kWarpsPerBlock * 32)
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 6)
 k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   extern __shared__ __align__(16) int32_t sm[];
   __shared__ int32_t s_slack[kMaxR];
@@ -1074,10 +1119,14 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   int32_t* sg_base = sg_ord + segcap;                   // [segcap] row - ordinal
   int32_t* sg_rank = sg_base + segcap;                  // [segcap] destination rank
   int32_t* base0 = sg_rank + (PASS > 0 ? segcap : 0);   // [E]
-  const int per_warp = E + 1 + (PASS > 0 ? R + (kPlanSubT * K + 3) / 4 : 0);
+  const int nsa = kPlanSubT * K;                        // assignments per sub-chunk
+  const bool pk = assign_packed(d);                     // expert and ordinal in one word
+  const int per_warp = E + 1 + nsa + (pk ? 0 : (nsa + 1) / 2) + (PASS > 0 ? R + (nsa + 3) / 4 : 0);
   int32_t* run = base0 + E + warp * per_warp;           // [E+1] running ordinals
-  int32_t* wrun = run + E + 1;                          // [R] running shared ordinals
-  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);   // [kPlanSubT*K] destination ranks
+  int32_t* so = run + E + 1;                            // [nsa] ordinals (| expert << 21)
+  uint16_t* se = reinterpret_cast<uint16_t*>(so + nsa); // [nsa] experts (E: dropped), !pk
+  int32_t* wrun = so + nsa + (pk ? 0 : (nsa + 1) / 2);  // [R] running shared ordinals
+  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);   // [nsa] destination ranks
 
   // The first batch of ids is an input no kernel of the plan writes: fetch it
   // before waiting for the predecessor grid.
@@ -1096,7 +1145,9 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   // solve passed its own wait and triggered the rerouting, whose trigger
   // launched this grid, so its block and sub-chunk counts are complete here.
   // The exclusive base of the block's first sub-chunk (earlier blocks of this
-  // rank), then each warp's running counts (plus the block's earlier warps).
+  // rank), then each warp's running counts (plus the block's earlier warps),
+  // then the warp's ordinals.  On a plan of one layer this overlaps the solve,
+  // which occupies a few SMs and leaves the rest to these blocks.
   for (int e = tid; e < E; e += nthr) base0[e] = 0;
   __syncthreads();
   const int32_t* cnt_r = s.sub_cnt + (int64_t)r * d.nsub * E;
@@ -1130,6 +1181,8 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
       run[e] = acc;
     }
     if (lane == 0) run[E] = 0;
+    __syncwarp();
+    assign_ordinals(ids + rbase, run, a0, a1, E, lane, lanemask_lt(), pk, v, so, se);
   }
   pdl_wait();
 
@@ -1161,27 +1214,47 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     int off = incl - local;
     for (int w = 0; w < warp; ++w) off += s_wsum[w];
     if (tid == nthr - 1) s_total = off + local;
+    // Per expert, for now: {first slot in the table, segment count, first
+    // segment in the rerouting's list}.  Then every segment is copied by a
+    // flat loop (its expert found by binary search over the first slots), so
+    // an expert with many segments costs no chain of dependent loads.
 #pragma unroll
     for (int u = 0; u < kExpPerThread; ++u) {
       const int e = eb + u;
       if (u < per && e < E) {
-        const int64_t gb = (int64_t)e * 3 * R + s0[u];
-        int4 g = make_int4(off, 0, 0, INT_MAX);
-        for (int j = 0; j < cnt[u] && off + j < segcap; ++j) {
-          const int ord = s.seg_ord[gb + j], rank = s.seg_rank[gb + j];
-          const int base = s.seg_base[gb + j];
-          sg_ord[off + j] = ord;
-          sg_base[off + j] = base;
-          if (PASS > 0) sg_rank[off + j] = rank;
-          if (j == 0) {
-            g.y = cnt[u] | (rank << 16);
-            g.z = base;
-          } else if (j == 1) {
-            g.w = ord;
-          }
+        sge[e] = make_int4(off, cnt[u], s0[u], 0);
+        off += cnt[u];
+      }
+    }
+    __syncthreads();
+    const int nseg = min(s_total, segcap);
+    for (int f = tid; f < nseg; f += nthr) {
+      int lo = 0, hi = E - 1;  // the last expert whose first slot is <= f
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sge[mid].x <= f) lo = mid; else hi = mid - 1;
+      }
+      const int4 h = sge[lo];
+      const int64_t gb = (int64_t)lo * 3 * R + h.z + (f - h.x);
+      sg_ord[f] = s.seg_ord[gb];
+      sg_base[f] = s.seg_base[gb];
+      if (PASS > 0) sg_rank[f] = s.seg_rank[gb];
+    }
+    __syncthreads();
+    // the 16-byte record: first segment, count | first rank << 16, first
+    // segment's row - ordinal, second segment's first ordinal (or INT_MAX)
+#pragma unroll
+    for (int u = 0; u < kExpPerThread; ++u) {
+      const int e = eb + u;
+      if (u < per && e < E) {
+        const int4 h = sge[e];
+        int4 g = make_int4(h.x, 0, 0, INT_MAX);
+        if (h.y > 0 && h.x < segcap) {
+          g.y = h.y | (PASS > 0 ? sg_rank[h.x] << 16 : 0);
+          g.z = sg_base[h.x];
+          if (h.y > 1 && h.x + 1 < segcap) g.w = sg_ord[h.x + 1];
         }
         sge[e] = g;
-        off += cnt[u];
       }
     }
     if (tid == 0) sge[E] = make_int4(0, 1, 0, INT_MAX);
@@ -1198,14 +1271,18 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   }
   if (!active) return;
 
-  // Main loop, 32 assignments per round: the stable ordinal of an assignment
-  // is its expert's running count plus its rank inside the round's match.any
-  // group (the group's leader advances the count).  The expert's segment record is fetched before the match, off the
-  // chain; dropped ids and lanes past the end share the dummy slot E.
+  // Each assignment's ordinal selects its segment and thus its row: the
+  // expert's segment record first (dropped ids share the dummy slot E).
   bool inconsistent = false;
   AssignCtx<PASS> c{sge, sg_ord, sg_base, sg_rank, L.dst_row + rbase,
-                    PASS > 0 ? s.asg_rank + rbase : nullptr, dr, a0, E, lane, lanemask_lt()};
-  assign_rounds<PASS>(c, ids + rbase, run, a0, a1, v, inconsistent);
+                    PASS > 0 ? s.asg_rank + rbase : nullptr, dr, a0, E, lane, 0u};
+  __syncwarp();
+#pragma unroll 4
+  for (int i = lane; i < a1 - a0; i += 32) {
+    const unsigned w = (unsigned)so[i];
+    const int e = pk ? (int)(w >> 21) : se[i], o = pk ? (int)(w & 0x1FFFFFu) : (int)w;
+    assign_finish<PASS>(c, sge[e], o, e < E, a0 + i, true, inconsistent);
+  }
   if (__any_sync(kFull, inconsistent) && lane == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
   if (PASS > 0) waterfill_subchunk(d, L, s, r, sub, t0, t1, dr, wrun, s_slack, s_W, lane);
 }
@@ -1827,7 +1904,9 @@ size_t solve_smem(const Dims& d) {
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
   const size_t segcap = (size_t)seg_capacity(d);
-  const size_t per_warp = (size_t)d.E + 1 + (pass > 0 ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
+  const size_t nsa = (size_t)kPlanSubT * d.K;
+  const size_t per_warp = (size_t)d.E + 1 + nsa + (assign_packed(d) ? 0 : (nsa + 1) / 2) +
+                          (pass > 0 ? d.R + (nsa + 3) / 4 : 0);
   return sizeof(int32_t) * (4 * ((size_t)d.E + 1) + segcap * (pass > 0 ? 3 : 2) + d.E +
                             (size_t)kWarpsPerBlock * per_warp);
 }
@@ -1853,14 +1932,30 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, 
 }  // namespace
 
 // Allow every kernel the device's opt-in shared-memory maximum once, so that
-// plans of any shape can coexist (each launch still requests only its own size).
+// plans of any shape can coexist (each launch still requests only its own size),
+// and prefer the largest shared-memory carveout for all of them.  The kernels of
+// one plan run side by side under programmatic dependent launch (the token
+// assignment's blocks compute their ordinals while the solve and the rerouting
+// run), and an SM configured with a smaller carveout for a kernel that needs
+// little shared memory could not take an assignment block until it drained.
+template <typename F>
+cudaError_t allow_plan_kernel(F* f, int max_smem) {
+  cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       (int)cudaSharedmemCarveoutMaxShared);
+  return e != cudaSuccess ? e : allow_max_dynamic_smem(f, max_smem);
+}
+template <typename F>
+cudaError_t prefer_max_carveout(F* f) {
+  return cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared);
+}
 template <int SMAX, bool PACK>
 cudaError_t allow_solve_pack(int max_smem) {
   cudaError_t e;
-  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 1, PACK>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 2, PACK>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_solve<SMAX, 3, PACK>, max_smem)) != cudaSuccess) return e;
-  return allow_max_dynamic_smem(k_solve<SMAX, 4, PACK>, max_smem);
+  if ((e = allow_plan_kernel(k_solve<SMAX, 1, PACK>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_solve<SMAX, 2, PACK>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_solve<SMAX, 3, PACK>, max_smem)) != cudaSuccess) return e;
+  return allow_plan_kernel(k_solve<SMAX, 4, PACK>, max_smem);
 }
 template <int SMAX>
 cudaError_t allow_solve(int max_smem) {
@@ -1874,14 +1969,32 @@ cudaError_t set_plan_attributes(int max_smem) {
   if ((e = allow_solve<2>(max_smem)) != cudaSuccess) return e;
   if ((e = allow_solve<4>(max_smem)) != cudaSuccess) return e;
   if ((e = allow_solve<8>(max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_hist, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_assign<0>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_assign<1>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_sample, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_sample_layout, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_sample_assign<0>, max_smem)) != cudaSuccess) return e;
-  if ((e = allow_max_dynamic_smem(k_wf_layer, max_smem)) != cudaSuccess) return e;
-  return allow_max_dynamic_smem(k_sample_assign<1>, max_smem);
+  if ((e = allow_plan_kernel(k_hist, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_assign<0>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_assign<1>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_sample, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_sample_layout, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_sample_assign<0>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_sample_assign<1>, max_smem)) != cudaSuccess) return e;
+  if ((e = allow_plan_kernel(k_wf_layer, max_smem)) != cudaSuccess) return e;
+  if ((e = prefer_max_carveout(k_reroute)) != cudaSuccess) return e;
+  if ((e = prefer_max_carveout(k_shared_scan)) != cudaSuccess) return e;
+  if ((e = prefer_max_carveout(k_fixup)) != cudaSuccess) return e;
+  return prefer_max_carveout(k_wf_layer_prep);
+}
+
+// The solve's dynamic shared memory: the whole of what the SM allows a block,
+// so that no other block shares the SM of a solve CTA.  Each cap candidate's
+// greedy is a serial chain of dependent steps; while it runs, the token
+// assignment's blocks compute their ordinals on every other SM, and on the
+// solve's SMs they would take issue slots from the chain.
+cudaError_t solve_launch_smem(const Dims& d, int max_smem, int* bytes) {
+  cudaFuncAttributes a;
+  const cudaError_t e = cudaFuncGetAttributes(&a, k_solve<1, 1, true>);
+  if (e != cudaSuccess) return e;
+  const size_t need = solve_smem(d), all = (size_t)max_smem - a.sharedSizeBytes;
+  *bytes = (int)(need > all ? need : all);
+  return cudaSuccess;
 }
 
 // The solve: a cluster of ceil(J / kSolveWarps) CTAs (one cap candidate per
@@ -1908,7 +2021,7 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), unsigned ctas, unsigned
 
 template <int SMAX>
 cudaError_t launch_solve_rw(const Dims& d, const LayerBuf& L, const Scratch& s, cudaStream_t st) {
-  const size_t ss = solve_smem(d);
+  const size_t ss = (size_t)d.solve_smem;
   const unsigned nt = kSolveThreads;
   const unsigned nc = (unsigned)((d.J + kSolveWarps - 1) / kSolveWarps);
   const int rw = (d.R + 31) / 32;

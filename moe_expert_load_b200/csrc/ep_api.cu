@@ -29,7 +29,7 @@ struct Layout {
       shared_rank, shared_row, cand, rep_list, rep_eptr, rep_nexp, rep_experts, inst_count, stats;
   size_t layer_bytes;
   // scratch (absolute)
-  size_t sub_cnt, blk_cnt, wsub_cnt, seg_ptr, seg_ord, seg_rank, seg_base, inst_rel, slack, wf, sbase,
+  size_t sub_cnt, blk_cnt, wsub_cnt, seg_rec, seg_ord, seg_rank, seg_base, inst_rel, slack, wf, sbase,
       shared_tot, asg_rank, smp_cum, smp_inst, smp_key, smp_sub, smp_blk, smp_row0, rank_rows,
       prev_base,
       acc_load, acc_misc, smp_tot;
@@ -123,7 +123,7 @@ Layout make_layout(const ep::Dims& d, int num_layers) {
   L.sub_cnt = s.take(i4 * (size_t)d.R * d.nsub * d.E);
   L.blk_cnt = s.take(i4 * (size_t)d.R * ((d.nsub + ep::kPlanWarps - 1) / ep::kPlanWarps) * d.E);
   L.wsub_cnt = s.take(d.sh ? i4 * (size_t)d.R * d.R * d.nsub : 0);
-  L.seg_ptr = s.take(i4 * (size_t)d.E * (d.R + 1));
+  L.seg_rec = s.take(i4 * 8 * (size_t)d.R * d.E);
   L.seg_ord = s.take(i4 * (size_t)d.E * 3 * d.R);
   L.seg_rank = s.take(i4 * (size_t)d.E * 3 * d.R);
   L.seg_base = s.take(i4 * (size_t)d.E * 3 * d.R);
@@ -205,7 +205,7 @@ ep::Scratch scratch(const ep_plan* p) {
   s.sub_cnt = at(p, l.sub_cnt);
   s.blk_cnt = at(p, l.blk_cnt);
   s.wsub_cnt = p->d.sh ? at(p, l.wsub_cnt) : nullptr;
-  s.seg_ptr = at(p, l.seg_ptr);
+  s.seg_rec = at(p, l.seg_rec);
   s.seg_ord = at(p, l.seg_ord);
   s.seg_rank = at(p, l.seg_rank);
   s.seg_base = at(p, l.seg_base);

@@ -66,7 +66,8 @@ struct Scratch {
   int32_t* sub_cnt;   // [R][nsub][E] per-sub-chunk counts
   int32_t* blk_cnt;   // [R][ceil(nsub/kPlanWarps)][E] per-block counts
   int32_t* wsub_cnt;  // [R][R*nsub] shared-slot counts per (dest rank, sub-chunk), then bases
-  int32_t* seg_ptr;   // [E][R+1] first segment of each source rank, per expert
+  int32_t* seg_rec;   // [R][E][8] per (source rank, expert): the first two segments
+                      // and where the third begins, as two int4 records
   int32_t* seg_ord;   // [E][3R] first ordinal of the segment
   int32_t* seg_rank;  // [E][3R] destination rank
   int32_t* seg_base;  // [E][3R] first row minus first ordinal: absolute without a shared

@@ -628,7 +628,9 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
 // own rank up to its quota; the residual demands, laid end to end in source
 // order, fill the residual quotas laid end to end in instance order.  The
 // output is, per (expert, source), the ordered segments (first ordinal,
-// destination rank, first row relative to that rank's block).
+// destination rank, first row minus first ordinal), and per (source, expert) a
+// 32-byte record of the first two segments that the token assignment copies
+// with one coalesced load.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBuf L, Scratch s) {
   __shared__ int32_t s_irank[kWarpsPerBlock][kMaxR];  // instance j: rank
@@ -828,7 +830,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
       segbase[k] = carry + incl - cnt[k];
       carry += __shfl_sync(kFull, incl, 31);
     }
-    if (lane == 0) s.seg_ptr[e * (R + 1) + R] = carry;
   }
   // pass 2: write the segments
   int32_t* sord = s.seg_ord + (int64_t)e * 3 * R;
@@ -841,15 +842,34 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   for (int k = 0; k < kRW; ++k) {
     const int r = lane + 32 * k;
     if (r >= R) continue;
-    s.seg_ptr[e * (R + 1) + r] = segbase[k];
     int w = segbase[k];
+    // the record of (r, e) for the token assignment: {first segment's index in
+    // the lists, count | first rank << 16, first row base, second segment's
+    // first ordinal} and {second rank, second row base, third segment's first
+    // ordinal}; ordinals past the lists' end never occur
+    int4 r0 = make_int4(e * 3 * R + w, cnt[k], 0, INT_MAX);
+    int4 r1 = make_int4(0, 0, INT_MAX, 0);
+    auto put = [&](int ord, int rank, int base) {
+      const int i = w - segbase[k];
+      if (i == 0) {
+        r0.y |= rank << 16;
+        r0.z = base;
+      } else if (i == 1) {
+        r0.w = ord;
+        r1.x = rank;
+        r1.y = base;
+      } else if (i == 2) {
+        r1.z = ord;
+      }
+      sord[w] = ord;
+      srank[w] = rank;
+      sbase[w] = base;
+      ++w;
+    };
     if (locr[k] > 0) {
       const int j = jof[r];
       const int before = min(max(PD[k] - ipq[j], 0), iq[j]);  // remote rows of earlier sources
-      sord[w] = 0;
-      srank[w] = r;
-      sbase[w] = (absolute ? s_rb[r] : 0) + irel[j] + before;
-      ++w;
+      put(0, r, (absolute ? s_rb[r] : 0) + irel[j] + before);
     }
     if (Dr[k] > 0) {
       const int end = PD[k] + Dr[k];
@@ -858,12 +878,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
         const int lo = max(PD[k], ipq[j]);
         const int c = irank[j];
         const int ord = locr[k] + (lo - PD[k]);
-        sord[w] = ord;
-        srank[w] = c;
-        sbase[w] = (absolute ? s_rb[c] : 0) + irel[j] + (c < r ? iloc[j] : 0) + (lo - ipq[j]) - ord;
-        ++w;
+        put(ord, c, (absolute ? s_rb[c] : 0) + irel[j] + (c < r ? iloc[j] : 0) + (lo - ipq[j]) - ord);
       }
     }
+    int4* rec = reinterpret_cast<int4*>(s.seg_rec) + ((int64_t)r * E + e) * 2;
+    rec[0] = r0;
+    rec[1] = r1;
   }
 }
 
@@ -986,15 +1006,14 @@ __device__ __forceinline__ void waterfill_subchunk(const Dims& d, const LayerBuf
 
 // ---------------------------------------------------------------------------
 // a4 (+a5): token assignment.  A block owns up to 8 consecutive sub-chunks of
-// one source rank r (one per warp).  It first copies rank r's rerouting
-// segments into shared memory — for each segment (first ordinal, row offset,
-// destination rank), and per expert one 16-byte record holding its first
-// segment and where the second begins, so that most lookups are one load —
-// and the exclusive base of its first sub-chunk, the sum of the rank's earlier
-// blocks' totals.  The stable ordinal of (t, k) among rank r's assignments of
-// expert e = that base + the counts of the block's earlier warps + the warp's
-// running count + the rank inside the 32-lane match.any group; the ordinal
-// selects the segment and thus the row.
+// one source rank r (one per warp).  The stable ordinal of (t, k) among rank
+// r's assignments of expert e = the counts of the rank's earlier blocks + those
+// of the block's earlier warps + the warp's running count + the rank inside
+// the 32-lane match.any group; these need only the ids and the histogram, so
+// the block computes them before waiting for the rerouting (while the solve
+// runs).  After the wait it copies rank r's per-expert segment records (the
+// first two segments and where the third begins) into shared memory, and each
+// ordinal selects its segment and thus its row.
 // PASS 0 (no shared expert): rows.  PASS 1 (shared expert): rows relative to
 // the destination rank's block and the destination ranks, then the Waterfill
 // pick of every token, its ordinal among the sub-chunk's tokens with that pick,
@@ -1007,47 +1026,48 @@ __host__ __device__ __forceinline__ bool assign_packed(const Dims& d) {
   return (int64_t)d.T * d.K <= ((int64_t)1 << 21);
 }
 
-__host__ __device__ __forceinline__ int seg_capacity(const Dims& d) {
-  // per source rank: at most one local segment per expert, and the remote
-  // overlaps of an expert are at most its number of instances
-  return 2 * d.E + d.R * d.S + 1;
-}
-
 template <int PASS>
 struct AssignCtx {
-  const int4* sge;       // [E+1] per-expert first-segment records (slot E: dummy)
-  const int32_t* sg_ord;
-  const int32_t* sg_base;
-  const int32_t* sg_rank;
+  const int4* sge;       // [E+1] per-expert records of the first two segments (slot E: dummy)
+  const int4* rec1;      // [E] the second segment and where the third begins
+  const int32_t* gord;   // the rerouting's segment lists in global memory
+  const int32_t* gbase;
+  const int32_t* grk;
   int32_t* drow;         // dst_row of the source rank
   uint8_t* grank;        // destination-rank bytes of the source rank (PASS 1)
   uint8_t* dr;           // the sub-chunk's destination ranks in shared memory (PASS 1)
-  int a0, E, lane;
-  unsigned lt;           // lanes below this one
+  int a0, E;
 };
 
-// The row (and destination rank) of ordinal o of an expert whose first-segment
-// record is g; ok is false for a dropped id or an expert without segments.
+// The row (and destination rank) of ordinal o of expert e; ok is false for a
+// dropped id or an expert without segments.  The segment is the last one that
+// starts at or before o: the first two are in shared memory, a third or later
+// one (rare: a source rank's demand spread over several remote instances) is
+// found in the rerouting's list in global memory.
 template <int PASS>
-__device__ __forceinline__ void assign_finish(const AssignCtx<PASS>& c, const int4& g, int o,
-                                              bool valid, int idx, bool in, bool& inconsistent) {
+__device__ __forceinline__ void assign_finish(const AssignCtx<PASS>& c, int e, int o, bool valid,
+                                              int idx, bool& inconsistent) {
+  const int4 g = c.sge[e];
   const int n = g.y & 0xffff;
   int b = g.z, q = g.y >> 16;
-  if (o >= g.w) {  // a later segment: the last one starting at or before o
-    int si = g.x + n - 1;
-    while (si > g.x && c.sg_ord[si] > o) --si;
-    b = c.sg_base[si];
-    if (PASS > 0) q = c.sg_rank[si];
+  if (o >= g.w) {
+    const int4 h = c.rec1[e];
+    b = h.y;
+    q = h.x;
+    if (o >= h.z) {
+      int si = g.x + n - 1;
+      while (si > g.x + 2 && c.gord[si] > o) --si;
+      b = c.gbase[si];
+      if (PASS > 0) q = c.grk[si];
+    }
   }
   const bool ok = valid && n > 0;
   inconsistent |= valid && n == 0;
-  if (in) {
-    c.drow[idx] = ok ? b + o : -1;
-    if (PASS > 0) {
-      const uint8_t rank = ok ? (uint8_t)q : (uint8_t)kNoRank;
-      c.dr[idx - c.a0] = rank;
-      c.grank[idx] = rank;
-    }
+  c.drow[idx] = ok ? b + o : -1;
+  if (PASS > 0) {
+    const uint8_t rank = ok ? (uint8_t)q : (uint8_t)kNoRank;
+    c.dr[idx - c.a0] = rank;
+    c.grank[idx] = rank;
   }
 }
 
@@ -1100,8 +1120,6 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   extern __shared__ __align__(16) int32_t sm[];
   __shared__ int32_t s_slack[kMaxR];
   __shared__ int32_t s_W[kMaxR];
-  __shared__ int32_t s_wsum[kWarpsPerBlock];
-  __shared__ int32_t s_total;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nthr = blockDim.x;
   const int R = d.R, E = d.E, K = d.K;
   const int nbpr = (d.nsub + kWarpsPerBlock - 1) / kWarpsPerBlock;
@@ -1109,16 +1127,12 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   const int sub0 = (blockIdx.x - r * nbpr) * kWarpsPerBlock;
   const int sub = sub0 + warp;
   const bool active = sub < d.nsub;
-  const int segcap = seg_capacity(d);
-  // per expert: {first segment, segment count | first segment's rank << 16,
-  // first segment's row - ordinal, second segment's first ordinal (or INT_MAX)}
-  // slot E of the record table and of the running counts is a dummy that
-  // dropped ids (and lanes past the end of the sub-chunk) share
+  // the rerouting's records of source rank r (see k_reroute); slot E of the
+  // first table and of the running counts is a dummy that dropped ids (and
+  // lanes past the end of the sub-chunk) share
   int4* sge = reinterpret_cast<int4*>(sm);              // [E+1]
-  int32_t* sg_ord = sm + 4 * (E + 1);                   // [segcap] first ordinal
-  int32_t* sg_base = sg_ord + segcap;                   // [segcap] row - ordinal
-  int32_t* sg_rank = sg_base + segcap;                  // [segcap] destination rank
-  int32_t* base0 = sg_rank + (PASS > 0 ? segcap : 0);   // [E]
+  int4* rec1 = sge + E + 1;                             // [E]
+  int32_t* base0 = reinterpret_cast<int32_t*>(rec1 + E);  // [E]
   const int nsa = kPlanSubT * K;                        // assignments per sub-chunk
   const bool pk = assign_packed(d);                     // expert and ordinal in one word
   const int per_warp = E + 1 + nsa + (pk ? 0 : (nsa + 1) / 2) + (PASS > 0 ? R + (nsa + 3) / 4 : 0);
@@ -1186,76 +1200,13 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   }
   pdl_wait();
 
-  // rank r's segment table (the rerouting's output)
+  // rank r's segment records (the rerouting's output), and with a shared
+  // expert the Waterfill slack and loads
   {
-    const int per = (E + nthr - 1) / nthr;
-    const int eb = tid * per;
-    int cnt[kExpPerThread], s0[kExpPerThread], local = 0;
-#pragma unroll
-    for (int u = 0; u < kExpPerThread; ++u) {
-      const int e = eb + u;
-      cnt[u] = 0;
-      s0[u] = 0;
-      if (u < per && e < E) {
-        const int sp = e * (R + 1) + r;
-        s0[u] = s.seg_ptr[sp];
-        cnt[u] = s.seg_ptr[sp + 1] - s0[u];
-      }
-      local += cnt[u];
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    int off = incl - local;
-    for (int w = 0; w < warp; ++w) off += s_wsum[w];
-    if (tid == nthr - 1) s_total = off + local;
-    // Per expert, for now: {first slot in the table, segment count, first
-    // segment in the rerouting's list}.  Then every segment is copied by a
-    // flat loop (its expert found by binary search over the first slots), so
-    // an expert with many segments costs no chain of dependent loads.
-#pragma unroll
-    for (int u = 0; u < kExpPerThread; ++u) {
-      const int e = eb + u;
-      if (u < per && e < E) {
-        sge[e] = make_int4(off, cnt[u], s0[u], 0);
-        off += cnt[u];
-      }
-    }
-    __syncthreads();
-    const int nseg = min(s_total, segcap);
-    for (int f = tid; f < nseg; f += nthr) {
-      int lo = 0, hi = E - 1;  // the last expert whose first slot is <= f
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (sge[mid].x <= f) lo = mid; else hi = mid - 1;
-      }
-      const int4 h = sge[lo];
-      const int64_t gb = (int64_t)lo * 3 * R + h.z + (f - h.x);
-      sg_ord[f] = s.seg_ord[gb];
-      sg_base[f] = s.seg_base[gb];
-      if (PASS > 0) sg_rank[f] = s.seg_rank[gb];
-    }
-    __syncthreads();
-    // the 16-byte record: first segment, count | first rank << 16, first
-    // segment's row - ordinal, second segment's first ordinal (or INT_MAX)
-#pragma unroll
-    for (int u = 0; u < kExpPerThread; ++u) {
-      const int e = eb + u;
-      if (u < per && e < E) {
-        const int4 h = sge[e];
-        int4 g = make_int4(h.x, 0, 0, INT_MAX);
-        if (h.y > 0 && h.x < segcap) {
-          g.y = h.y | (PASS > 0 ? sg_rank[h.x] << 16 : 0);
-          g.z = sg_base[h.x];
-          if (h.y > 1 && h.x + 1 < segcap) g.w = sg_ord[h.x + 1];
-        }
-        sge[e] = g;
-      }
+    const int4* rec = reinterpret_cast<const int4*>(s.seg_rec) + (int64_t)r * E * 2;
+    for (int i = tid; i < 2 * E; i += nthr) {
+      const int4 x = rec[i];
+      if (i & 1) rec1[i >> 1] = x; else sge[i >> 1] = x;
     }
     if (tid == 0) sge[E] = make_int4(0, 1, 0, INT_MAX);
   }
@@ -1265,23 +1216,19 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
       s_W[q] = L.W[q];
     }
   __syncthreads();
-  if (s_total > segcap) {
-    if (tid == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
-    return;
-  }
   if (!active) return;
 
   // Each assignment's ordinal selects its segment and thus its row: the
   // expert's segment record first (dropped ids share the dummy slot E).
   bool inconsistent = false;
-  AssignCtx<PASS> c{sge, sg_ord, sg_base, sg_rank, L.dst_row + rbase,
-                    PASS > 0 ? s.asg_rank + rbase : nullptr, dr, a0, E, lane, 0u};
+  AssignCtx<PASS> c{sge, rec1, s.seg_ord, s.seg_base, s.seg_rank, L.dst_row + rbase,
+                    PASS > 0 ? s.asg_rank + rbase : nullptr, dr, a0, E};
   __syncwarp();
 #pragma unroll 4
   for (int i = lane; i < a1 - a0; i += 32) {
     const unsigned w = (unsigned)so[i];
     const int e = pk ? (int)(w >> 21) : se[i], o = pk ? (int)(w & 0x1FFFFFu) : (int)w;
-    assign_finish<PASS>(c, sge[e], o, e < E, a0 + i, true, inconsistent);
+    assign_finish<PASS>(c, e, o, e < E, a0 + i, inconsistent);
   }
   if (__any_sync(kFull, inconsistent) && lane == 0) atomicOr(&L.stats->status, EP_DEV_INCONSISTENT);
   if (PASS > 0) waterfill_subchunk(d, L, s, r, sub, t0, t1, dr, wrun, s_slack, s_W, lane);
@@ -1903,11 +1850,10 @@ size_t solve_smem(const Dims& d) {
 }
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {
-  const size_t segcap = (size_t)seg_capacity(d);
   const size_t nsa = (size_t)kPlanSubT * d.K;
   const size_t per_warp = (size_t)d.E + 1 + nsa + (assign_packed(d) ? 0 : (nsa + 1) / 2) +
                           (pass > 0 ? d.R + (nsa + 3) / 4 : 0);
-  return sizeof(int32_t) * (4 * ((size_t)d.E + 1) + segcap * (pass > 0 ? 3 : 2) + d.E +
+  return sizeof(int32_t) * (4 * ((size_t)d.E + 1) + 4 * (size_t)d.E + d.E +
                             (size_t)kWarpsPerBlock * per_warp);
 }
 

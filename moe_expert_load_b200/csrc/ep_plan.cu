@@ -1450,9 +1450,16 @@ __global__ void __launch_bounds__(kLayoutThreads) k_sample_layout(Dims d, LayerB
 // kappa is the first row of (r, kappa) plus its ordinal among rank r's
 // assignments with that key in (t, k) order: the counts of the rank's earlier
 // blocks and the block's earlier warps, the warp's running count and the rank
-// inside the 32-lane match.any group.  SH: rows relative to the destination
-// rank's block and the destination rank bytes, then the Waterfill picks
+// inside the 32-lane match.any group.  The ordinals need only the draws, so
+// they are computed before the wait (while the layout kernel runs); after it
+// the first rows are added.  SH: rows relative to the destination rank's block
+// and the destination rank bytes, then the Waterfill picks
 // (waterfill_subchunk), exactly as k_assign<1>.
+__host__ __device__ __forceinline__ bool sample_assign_packed(const Dims& d) {
+  // ordinal and key (< 2^12 with the dummy) in one word
+  return (int64_t)d.T * d.K <= ((int64_t)1 << 20);
+}
+
 template <int SH>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
 k_sample_assign(Dims d, LayerBuf L, Scratch s) {
@@ -1470,10 +1477,14 @@ k_sample_assign(Dims d, LayerBuf L, Scratch s) {
   int32_t* s_row0 = sm;                        // [NK] first row of (r, key)
   int32_t* s_krank = s_row0 + NK;              // [NK] destination rank of the key (SH)
   int32_t* base0 = s_krank + (SH ? NK : 0);    // [NK] draws of the rank's earlier blocks
-  const int per_warp = NK + (SH ? R + (kPlanSubT * K + 3) / 4 : 0);
+  const int nsa = kPlanSubT * K;
+  const bool pk = sample_assign_packed(d);
+  const int per_warp = NK + nsa + (pk ? 0 : (nsa + 1) / 2) + (SH ? R + (nsa + 3) / 4 : 0);
   int32_t* run = base0 + NK + warp * per_warp; // [NK] running ordinals
-  int32_t* wrun = run + NK;                    // [R] running shared ordinals (SH)
-  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);  // [kPlanSubT*K] ranks (SH)
+  int32_t* so = run + NK;                      // [nsa] ordinals (| key << 20)
+  uint16_t* sk = reinterpret_cast<uint16_t*>(so + nsa);  // [nsa] keys (!pk)
+  int32_t* wrun = so + nsa + (pk ? 0 : (nsa + 1) / 2);   // [R] running shared ordinals (SH)
+  uint8_t* dr = reinterpret_cast<uint8_t*>(wrun + R);    // [nsa] ranks (SH)
   pdl_trigger();
   // Before waiting: the draws (the sampling pass had completed before the
   // layout passed its own wait and launched this grid) — the exclusive base
@@ -1511,6 +1522,40 @@ k_sample_assign(Dims d, LayerBuf L, Scratch s) {
       run[k] = acc;
     }
   }
+  const int t0 = active ? sub * kPlanSubT : 0, t1 = active ? min(d.T, t0 + kPlanSubT) : 0;
+  const int a0 = t0 * K, a1 = t1 * K;
+  const int64_t rbase = (int64_t)r * d.T * K;
+  if (active) {
+    __syncwarp();
+    for (int a = a0; a < a1; a += kAsgBatch * 32) {
+      int v[kAsgBatch];
+#pragma unroll
+      for (int u = 0; u < kAsgBatch; ++u) {
+        const int idx = a + u * 32 + lane;
+        v[u] = idx < a1 ? (int)s.smp_key[rbase + idx] : 0xFFFF;
+      }
+#pragma unroll
+      for (int u = 0; u < kAsgBatch; ++u) {
+        if (a + u * 32 >= a1) break;
+        const int idx = a + u * 32 + lane;
+        const int key = v[u] < nk ? v[u] : nk;  // nk: a dropped id
+        const unsigned peers = match_bits(key, 32 - __clz(nk));
+        const int rk = __popc(peers & lanemask_lt());
+        const int o = key < nk ? run[key] + rk : 0;
+        __syncwarp();
+        if (key < nk && lane == __ffs(peers) - 1) run[key] = o + __popc(peers);
+        __syncwarp();
+        if (idx < a1) {
+          if (pk) {
+            so[idx - a0] = (int32_t)((unsigned)o | ((unsigned)key << 20));
+          } else {
+            so[idx - a0] = o;
+            sk[idx - a0] = (uint16_t)key;
+          }
+        }
+      }
+    }
+  }
   pdl_wait();
   for (int k = tid; k < nk; k += nthr) s_row0[k] = s.smp_row0[r * NK + k];
   if (SH)
@@ -1520,35 +1565,16 @@ k_sample_assign(Dims d, LayerBuf L, Scratch s) {
     }
   __syncthreads();
   if (!active) return;
-  const int t0 = sub * kPlanSubT, t1 = min(d.T, t0 + kPlanSubT);
-  const int a0 = t0 * K, a1 = t1 * K;
-  const int64_t rbase = (int64_t)r * d.T * K;
-  for (int a = a0; a < a1; a += kAsgBatch * 32) {
-    int v[kAsgBatch];
-#pragma unroll
-    for (int u = 0; u < kAsgBatch; ++u) {
-      const int idx = a + u * 32 + lane;
-      v[u] = idx < a1 ? (int)s.smp_key[rbase + idx] : 0xFFFF;
-    }
-#pragma unroll
-    for (int u = 0; u < kAsgBatch; ++u) {
-      if (a + u * 32 >= a1) break;
-      const int idx = a + u * 32 + lane;
-      const int key = v[u] < nk ? v[u] : -1;
-      const unsigned peers = match_bits(key >= 0 ? key : nk, 32 - __clz(nk));
-      const int rk = __popc(peers & lanemask_lt());
-      const int o = key >= 0 ? run[key] + rk : 0;
-      __syncwarp();
-      if (key >= 0 && lane == __ffs(peers) - 1) run[key] = o + __popc(peers);
-      __syncwarp();
-      if (idx < a1) {
-        L.dst_row[rbase + idx] = key >= 0 ? s_row0[key] + o : -1;
-        if (SH) {
-          const uint8_t q = key >= 0 ? (uint8_t)s_krank[key] : (uint8_t)kNoRank;
-          dr[idx - a0] = q;
-          s.asg_rank[rbase + idx] = q;
-        }
-      }
+#pragma unroll 4
+  for (int i = lane; i < a1 - a0; i += 32) {
+    const unsigned w = (unsigned)so[i];
+    const int key = pk ? (int)(w >> 20) : sk[i], o = pk ? (int)(w & 0xFFFFFu) : (int)w;
+    const bool ok = key < nk;
+    L.dst_row[rbase + a0 + i] = ok ? s_row0[key] + o : -1;
+    if (SH) {
+      const uint8_t q = ok ? (uint8_t)s_krank[key] : (uint8_t)kNoRank;
+      dr[i] = q;
+      s.asg_rank[rbase + a0 + i] = q;
     }
   }
   if (SH) {
@@ -1838,7 +1864,9 @@ size_t sample_layout_smem(const Dims& d) {
   return sizeof(int32_t) * (2 * (size_t)d.nkey + 2 * (size_t)d.R * d.G);
 }
 size_t sample_assign_smem(const Dims& d) {
-  const size_t per_warp = d.nkey + (d.sh ? d.R + (kPlanSubT * d.K + 3) / 4 : 0);
+  const size_t nsa = (size_t)kPlanSubT * d.K;
+  const size_t per_warp = d.nkey + nsa + (sample_assign_packed(d) ? 0 : (nsa + 1) / 2) +
+                          (d.sh ? d.R + (nsa + 3) / 4 : 0);
   return sizeof(int32_t) *
          ((size_t)d.nkey * (d.sh ? 3 : 2) + (size_t)kWarpsPerBlock * per_warp);
 }

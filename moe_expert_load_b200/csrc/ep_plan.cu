@@ -225,12 +225,14 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   int32_t* Qn_all = sm + d.E;     // [kSolveWarps][E]: this CTA's candidates' native quotas
   int32_t* cnt_e = Qn_all + kSolveWarps * d.E;  // [E+1]
   int32_t* s_rel = cnt_e + d.E + 1;     // [R*G] rank-relative first rows
+  int32_t* s_iex = s_rel + d.R * d.G;   // [R*G] the winner's instance table: experts
+  int32_t* s_iqu = s_iex + d.R * d.G;   // [R*G] and quotas
   __shared__ int32_t s_W0[kMaxR];
   __shared__ int32_t s_Wf[kMaxR];
   __shared__ int32_t s_se[kMaxR * kMaxS];
   __shared__ int32_t s_sq[kMaxR * kMaxS];
   __shared__ int32_t s_cmax[kMaxJ], s_crep[kMaxJ], s_cstop[kMaxJ];
-  __shared__ int32_t s_best, s_A, s_iter_cap_hit, s_tight, s_any_cap;
+  __shared__ int32_t s_best, s_A, s_iter_cap_hit, s_tight, s_any_cap, s_bmax;
   __shared__ int32_t s_base[kMaxR + 1];
   __shared__ int32_t s_wsum[kMaxJ];
 
@@ -247,6 +249,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   // histogram's load matrix before waiting for the solve
   pdl_wait();
   pdl_trigger();
+  const int hist_status = s.acc_misc[0];  // the histogram's status bits of this call
   // expert totals: the load matrix's columns summed over source ranks (the
   // histogram adds only into the load matrix: one total per expert would
   // take an atomic from every block of the grid).  CTA c of the cluster sums
@@ -283,19 +286,14 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
     Tot[e] = *cluster.map_shared_rank(&Tot[e], c);
   }
   __syncthreads();
-  if (crank == 0) {
-    for (int e = tid; e < E; e += nthr) L.expert_total[e] = Tot[e];
-    if (tid == 0) {
-      L.stats->status = s.acc_misc[0];  // the first status bits of this call
-      s.acc_misc[0] = 0;
-    }
-  }
+  // (the totals, W0 and the statistics reach global memory only in the
+  // winner's last phase: no global store is queued ahead of the greedy's
+  // shared-memory loads)
   if (tid < R) {
     const int f = tid * eb + min(tid, er), n = eb + (tid < er ? 1 : 0);
     int w = 0;
     for (int i = 0; i < n; ++i) w += Tot[f + i];
     s_W0[tid] = w;
-    if (crank == 0) L.W0[tid] = w;
   }
   __syncthreads();
   if (warp == 0) {
@@ -308,7 +306,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
     bm = (int)__reduce_max_sync(kFull, (unsigned)bm);
     if (lane == 0) {
       s_A = a;
-      if (crank == 0) L.stats->before_max = bm;
+      s_bmax = bm;
     }
   }
   __syncthreads();
@@ -480,35 +478,32 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   // CTA lays the plan out
   cluster.sync();
   if (crank != s_best / kSolveWarps) return;
+  __shared__ int32_t s_wst[4];  // the winner's stop reason, replicas, cap, max load
   if (solver && j == s_best) {
+    if (lane == 0) {
+      s_wst[0] = stop;
+      s_wst[1] = replicas;
+      s_wst[2] = C;
+      s_wst[3] = maxW;
+    }
 #pragma unroll
     for (int k = 0; k < RW; ++k) {
       const int q = lane + 32 * k;
       if (q < R) {
         s_Wf[q] = Wr[k];
-        L.W[q] = Wr[k];
-        s.rank_rows[q] = Wr[k];  // routed rows per rank (the sampled mode recounts them)
 #pragma unroll
         for (int t = 0; t < SMAX; ++t)
           if (t < S) { s_se[q * S + t] = se[k][t]; s_sq[q * S + t] = sq[k][t]; }
       }
     }
-    if (lane == 0) {
-      ep_layer_stats* st = L.stats;
-      st->cap_idx = j;
-      st->stop_reason = stop;
-      st->tight_stop_reason = s_tight;
-      st->replicas = replicas;
-      st->cap = C;
-      st->assignments = A;
-      st->after_max = maxW;
-      st->realized_max = maxW;
-      if (s_any_cap) atomicOr(&st->status, EP_DEV_ITER_CAP);
-    }
   }
   __syncthreads();
 
   // ---- emit the winner's instance table ----
+  // Everything is laid out in shared memory first and written to global
+  // memory in one last phase: measured with clock readings, a phase that
+  // read shared memory after another phase's global stores waited
+  // 1500-2700 cycles behind them, five times over.
   const int G = d.G, Gmax = d.Gmax;
   const int32_t* Qw = Qn_all + (s_best % kSolveWarps) * E;
   for (int i = tid; i < R * G; i += nthr) {
@@ -522,23 +517,16 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
     } else {
       ex = E;  // the shared-expert column
     }
-    L.inst_expert[i] = ex;
-    L.inst_quota[i] = qu;
+    s_iex[i] = ex;
+    s_iqu[i] = qu;
   }
   for (int i = tid; i <= E; i += nthr) cnt_e[i] = 0;
   __syncthreads();
   if (tid < R) {  // rank-relative first row of every instance
     int run = 0;
     for (int col = 0; col < G; ++col) {
-      s.inst_rel[tid * G + col] = run;
       s_rel[tid * G + col] = run;
-      int qu = 0;
-      if (col < Gmax) {
-        if (col < eb + (tid < er ? 1 : 0)) qu = Qw[tid * eb + min(tid, er) + col];
-      } else if (col < Gmax + S) {
-        qu = s_sq[tid * S + col - Gmax];
-      }
-      run += qu;
+      run += s_iqu[tid * G + col];
     }
   }
   for (int i = tid; i < R * S; i += nthr)
@@ -561,8 +549,76 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
     if (lane == 0) s_base[R] = carry;
   }
   __syncthreads();
+  // replica lists grouped by expert (CSR): the offsets rep_eptr and the list
+  // of replicated experts come from one block-wide exclusive scan of
+  // (replicas of e) | (e has replicas) << 16 — both sums stay below 2^16 —
+  // and k_reroute writes each expert's slots into its part of the list
+  constexpr int kIPT = (kMaxE + 1 + kSolveThreads - 1) / kSolveThreads;
+  int vals[kIPT], local = 0;
+#pragma unroll
+  for (int u = 0; u < kIPT; ++u) {
+    const int e = tid * kIPT + u;
+    const int c = e < E ? cnt_e[e] : 0;
+    vals[u] = c | (c > 0 ? 1 << 16 : 0);
+    local += vals[u];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = lane < nthr / 32 ? s_wsum[lane] : 0;
+    int wi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, wi, o);
+      if (lane >= o) wi += y;
+    }
+    if (lane < nthr / 32) s_wsum[lane] = wi - v;
+  }
+  __syncthreads();
+
+  // ---- the global writes ----
+  if (tid == 0) {
+    ep_layer_stats* st = L.stats;
+    st->status = hist_status | (s_any_cap ? EP_DEV_ITER_CAP : 0);
+    s.acc_misc[0] = 0;  // zero again for the next call
+    st->before_max = s_bmax;
+    st->cap_idx = s_best;
+    st->stop_reason = s_wst[0];
+    st->tight_stop_reason = s_tight;
+    st->replicas = s_wst[1];
+    st->cap = s_wst[2];
+    st->assignments = A;
+    st->after_max = s_wst[3];
+    st->realized_max = s_wst[3];
+  }
+  for (int e = tid; e < E; e += nthr) L.expert_total[e] = Tot[e];
+  for (int q = tid; q < R; q += nthr) {
+    L.W0[q] = s_W0[q];
+    L.W[q] = s_Wf[q];
+    s.rank_rows[q] = s_Wf[q];  // routed rows per rank (the sampled mode recounts them)
+  }
+  int run = s_wsum[warp] + incl - local;
+#pragma unroll
+  for (int u = 0; u < kIPT; ++u) {
+    const int e = tid * kIPT + u;
+    if (e <= E) L.rep_eptr[e] = run & 0xffff;
+    if (e < E && (vals[u] & 0xffff)) L.rep_experts[run >> 16] = e;
+    if (e == E) L.rep_nexp[0] = run >> 16;
+    run += vals[u];
+  }
+  for (int i = tid; i < R * G; i += nthr) {
+    L.inst_expert[i] = s_iex[i];
+    L.inst_quota[i] = s_iqu[i];
+    s.inst_rel[i] = s_rel[i];
+    if (!d.sh) L.inst_off[i] = s_base[i / G] + s_rel[i];
+  }
   if (!d.sh) {
-    for (int i = tid; i < R * G; i += nthr) L.inst_off[i] = s_base[i / G] + s_rel[i];
     if (tid == 0) L.inst_off[R * G] = s_base[R];
     for (int q = tid; q <= R; q += nthr) L.rank_base[q] = s_base[q];
     if (tid == 0) L.stats->rows = s_base[R];
@@ -576,49 +632,6 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
       s.wf[1] = (int)((H * d.bonus + 999) / 1000);
     }
     for (int q = tid; q < R; q += nthr) s.slack[q] = (int)max(H - (int64_t)s_Wf[q], (int64_t)0);
-  }
-  // replica lists grouped by expert (CSR): the offsets rep_eptr and the list
-  // of replicated experts come from one block-wide exclusive scan of
-  // (replicas of e) | (e has replicas) << 16 — both sums stay below 2^16 —
-  // and k_reroute writes each expert's slots into its part of the list
-  {
-    constexpr int kIPT = (kMaxE + 1 + kSolveThreads - 1) / kSolveThreads;
-    int vals[kIPT], local = 0;
-#pragma unroll
-    for (int u = 0; u < kIPT; ++u) {
-      const int e = tid * kIPT + u;
-      const int c = e < E ? cnt_e[e] : 0;
-      vals[u] = c | (c > 0 ? 1 << 16 : 0);
-      local += vals[u];
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) s_wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      const int v = lane < nthr / 32 ? s_wsum[lane] : 0;
-      int wi = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, wi, o);
-        if (lane >= o) wi += y;
-      }
-      if (lane < nthr / 32) s_wsum[lane] = wi - v;
-    }
-    __syncthreads();
-    int run = s_wsum[warp] + incl - local;
-#pragma unroll
-    for (int u = 0; u < kIPT; ++u) {
-      const int e = tid * kIPT + u;
-      if (e <= E) L.rep_eptr[e] = run & 0xffff;
-      if (e < E && (vals[u] & 0xffff)) L.rep_experts[run >> 16] = e;
-      if (e == E) L.rep_nexp[0] = run >> 16;
-      run += vals[u];
-    }
   }
 }
 
@@ -1874,7 +1887,8 @@ size_t wf_layer_smem(const Dims& d) {
   return sizeof(int32_t) * (size_t)kWarpsPerBlock * (d.R + (kPlanSubT * d.K + 3) / 4);
 }
 size_t solve_smem(const Dims& d) {
-  return sizeof(int32_t) * ((size_t)d.E * (1 + kSolveWarps) + ((size_t)d.E + 1) + (size_t)d.R * d.G);
+  return sizeof(int32_t) *
+         ((size_t)d.E * (1 + kSolveWarps) + ((size_t)d.E + 1) + 3 * (size_t)d.R * d.G);
 }
 size_t hist_smem(const Dims& d) { return sizeof(int32_t) * (size_t)kWarpsPerBlock * d.E; }
 size_t assign_smem(const Dims& d, int pass) {

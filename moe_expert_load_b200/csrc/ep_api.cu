@@ -12,7 +12,7 @@
 
 namespace ep {
 cudaError_t set_plan_attributes(int max_smem);
-cudaError_t solve_launch_smem(const Dims& d, int max_smem, int* bytes);
+cudaError_t plan_launch_shapes(Dims& d, int max_smem, int sms);
 cudaError_t set_copy_attributes(int max_smem);
 }  // namespace ep
 
@@ -92,6 +92,7 @@ ep_status_t make_dims(const ep_config* c, ep::Dims* d) {
   d->sseed = c->sampling_seed;
   d->nkey = E + R * d->S;  // at most 1024 + 128 * 8 keys: they fit the uint16 key buffer
   d->solve_smem = 0;       // set at plan creation, from the device's shared-memory limit
+  d->fix_grid = 1;         // set at plan creation, from the device's SM count
   return EP_OK;
 }
 
@@ -290,7 +291,12 @@ ep_status_t ep_plan_create(const ep_config* cfg, void* d_workspace, size_t works
   if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return EP_ERR_CUDA;
   if (ep::set_plan_attributes(max_smem) != cudaSuccess) return EP_ERR_CUDA;
-  if (ep::solve_launch_smem(d, max_smem, &d.solve_smem) != cudaSuccess) return EP_ERR_CUDA;
+  {
+    int dev_sms = 0;  // the device's own count: the plan kernels' grids are not overridden
+    if (cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return EP_ERR_CUDA;
+    if (ep::plan_launch_shapes(d, max_smem, dev_sms) != cudaSuccess) return EP_ERR_CUDA;
+  }
   if (ep::set_copy_attributes(max_smem) != cudaSuccess) return EP_ERR_CUDA;
   ep_plan* p = new (std::nothrow) ep_plan;
   if (!p) return EP_ERR_INVALID_ARGUMENT;

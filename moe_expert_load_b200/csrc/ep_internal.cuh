@@ -37,6 +37,7 @@ struct Dims {
   uint64_t sseed;    // seed of the sampled mode's per-assignment draw
   int nkey;          // sampled mode: key space E + R*S (expert-major instance keys)
   int solve_smem;    // dynamic shared memory of the solve launch (set at plan creation)
+  int fix_grid;      // blocks of the shared-slot fix-up: those resident at once (plan creation)
 };
 
 // One layer's slot in the plan cache (all device pointers).

@@ -1976,12 +1976,20 @@ cudaError_t set_plan_attributes(int max_smem) {
 // greedy is a serial chain of dependent steps; while it runs, the token
 // assignment's blocks compute their ordinals on every other SM, and on the
 // solve's SMs they would take issue slots from the chain.
-cudaError_t solve_launch_smem(const Dims& d, int max_smem, int* bytes) {
+//
+// The fix-up's grid: the blocks that are resident at once.  Its blocks wait
+// for the shared scan before their grid-stride loop, so a second wave of
+// blocks would start only as the first one leaves.
+cudaError_t plan_launch_shapes(Dims& d, int max_smem, int sms) {
   cudaFuncAttributes a;
-  const cudaError_t e = cudaFuncGetAttributes(&a, k_solve<1, 1, true>);
+  cudaError_t e = cudaFuncGetAttributes(&a, k_solve<1, 1, true>);
   if (e != cudaSuccess) return e;
   const size_t need = solve_smem(d), all = (size_t)max_smem - a.sharedSizeBytes;
-  *bytes = (int)(need > all ? need : all);
+  d.solve_smem = (int)(need > all ? need : all);
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_fixup, kFixThreads, 0);
+  if (e != cudaSuccess) return e;
+  d.fix_grid = (per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1);
   return cudaSuccess;
 }
 
@@ -2084,7 +2092,8 @@ cudaError_t launch_shared_layout(const Dims& d, const LayerBuf& L, const Scratch
   const int64_t work = A4 > N ? A4 : N;
   const int64_t fblk = (work + kFixThreads - 1) / kFixThreads;
   if (work > 0)
-    err = launch_pdl(k_fixup, (unsigned)(fblk < 2048 ? fblk : 2048), kFixThreads, 0, st, d, L, s);
+    err = launch_pdl(k_fixup, (unsigned)(fblk < d.fix_grid ? fblk : d.fix_grid), kFixThreads, 0, st,
+                     d, L, s);
   return err;
 }
 

@@ -73,7 +73,8 @@ constexpr int kAsgBatch = 8;   // ids per lane per pass in k_assign
 // ---------------------------------------------------------------------------
 // a1: load histogram.  A block owns up to 8 consecutive sub-chunks of
 // kPlanSubT tokens of one source rank, one per warp.  Each warp loads its whole
-// sub-chunk at once (at most 16 ids per lane) and counts it into a private
+// sub-chunk at once (for K <= 8 four 16-byte vectors of ids per lane, when the
+// rank's ids are 16-byte aligned; else 16 single ids) and counts it into a private
 // shared-memory histogram with shared atomic adds; the warp writes its row of
 // counts and the block writes the sum of its rows (the two levels of bases of
 // the stable ordinals, used by k_assign).  The block then adds its sum to the

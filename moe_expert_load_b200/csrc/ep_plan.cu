@@ -104,7 +104,7 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
     const int n = a1 - t0 * K;
     auto count = [&](int v, bool in) {
       if (!in) return;
-      if (v < 0 || v >= E) bad = 1;
+      if (v < 0 || v >= E) ++bad;
       else atomicAdd(&hist[v], 1);  // integer: order-independent
     };
     if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
@@ -163,7 +163,13 @@ k_hist(const int32_t* __restrict__ ids, Dims d, Scratch s) {
       blk[e] = csum[u];
     }
   }
-  if (__any_sync(kFull, bad) && lane == 0) atomicOr(&s.acc_misc[0], EP_DEV_BAD_ID);
+  // ids outside [0, E): the status bit, and their count, from which the solve
+  // takes the number of assignments without a reduction of its own
+  const int nbad = (int)__reduce_add_sync(kFull, (unsigned)bad);
+  if (nbad && lane == 0) {
+    atomicOr(&s.acc_misc[0], EP_DEV_BAD_ID);
+    atomicAdd(&s.acc_misc[2], nbad);
+  }
 #pragma unroll
   for (int u = 0; u < kExpPerThread; ++u) {
     const int e = threadIdx.x + u * blockDim.x;
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   __shared__ int32_t s_se[kMaxR * kMaxS];
   __shared__ int32_t s_sq[kMaxR * kMaxS];
   __shared__ int32_t s_cmax[kMaxJ], s_crep[kMaxJ], s_cstop[kMaxJ];
-  __shared__ int32_t s_best, s_A, s_iter_cap_hit, s_tight, s_any_cap, s_bmax;
+  __shared__ int32_t s_best, s_iter_cap_hit, s_tight, s_any_cap, s_bmax;
   __shared__ int32_t s_base[kMaxR + 1];
   __shared__ int32_t s_wsum[kMaxJ];
 
@@ -251,6 +257,8 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   pdl_wait();
   pdl_trigger();
   const int hist_status = s.acc_misc[0];  // the histogram's status bits of this call
+  // A: every assignment with an id in [0, E) (the histogram counts the others)
+  const int A = (int)((int64_t)R * d.T * d.K - s.acc_misc[2]);
   // expert totals: the load matrix's columns summed over source ranks (the
   // histogram adds only into the load matrix: one total per expert would
   // take an atomic from every block of the grid).  CTA c of the cluster sums
@@ -259,6 +267,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   // then reads the other CTAs' totals from their shared memory.
   const int e_lo = crank * E / ncta, e_hi = (crank + 1) * E / ncta, ne = e_hi - e_lo;
   for (int e = e_lo + tid; e < e_hi; e += nthr) Tot[e] = 0;
+  for (int e = tid; e <= E; e += nthr) cnt_e[e] = 0;  // the winner's replica counts, at the end
   if (tid == 0) s_iter_cap_hit = 0;
   __syncthreads();
   if (ne > 0) {
@@ -297,21 +306,6 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
     s_W0[tid] = w;
   }
   __syncthreads();
-  if (warp == 0) {
-    int a = 0, bm = 0;
-    for (int q = lane; q < R; q += 32) {
-      a += s_W0[q];
-      bm = max(bm, s_W0[q]);
-    }
-    a = __reduce_add_sync(kFull, a);
-    bm = (int)__reduce_max_sync(kFull, (unsigned)bm);
-    if (lane == 0) {
-      s_A = a;
-      s_bmax = bm;
-    }
-  }
-  __syncthreads();
-  const int A = s_A;
 
   // ---- one greedy run per warp: candidate j = crank * kSolveWarps + warp ----
   const int j = crank * kSolveWarps + warp;
@@ -502,42 +496,42 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
 
   // ---- emit the winner's instance table ----
   // Everything is laid out in shared memory first and written to global
-  // memory in one last phase: measured with clock readings, a phase that
-  // read shared memory after another phase's global stores waited
-  // 1500-2700 cycles behind them, five times over.
+  // memory in one last phase; the layout takes two barriers.  Thread q walks
+  // rank q's columns once (expert, quota, rank-relative first row, and the
+  // replica count of the column's expert); the last warp scans the ranks'
+  // routed rows into the ranks' first rows.  (With only the solve's four warps
+  // on the SM, each barrier-separated phase costs its full dependency chain:
+  // clock readings put the earlier five-phase layout at 0.8-1.6 us a phase.)
   const int G = d.G, Gmax = d.Gmax;
   const int32_t* Qw = Qn_all + (s_best % kSolveWarps) * E;
-  for (int i = tid; i < R * G; i += nthr) {
-    const int q = i / G, col = i - (i / G) * G;
-    int ex = -1, qu = 0;
-    if (col < Gmax) {
-      if (col < eb + (q < er ? 1 : 0)) { ex = q * eb + min(q, er) + col; qu = Qw[ex]; }
-    } else if (col < Gmax + S) {
-      ex = s_se[q * S + col - Gmax];
-      qu = s_sq[q * S + col - Gmax];
-    } else {
-      ex = E;  // the shared-expert column
-    }
-    s_iex[i] = ex;
-    s_iqu[i] = qu;
-  }
-  for (int i = tid; i <= E; i += nthr) cnt_e[i] = 0;
-  __syncthreads();
-  if (tid < R) {  // rank-relative first row of every instance
+  if (tid < R) {
+    const int q = tid, nf = q * eb + min(q, er), nn = eb + (q < er ? 1 : 0);
     int run = 0;
     for (int col = 0; col < G; ++col) {
-      s_rel[tid * G + col] = run;
-      run += s_iqu[tid * G + col];
+      int ex = -1, qu = 0;
+      if (col < Gmax) {
+        if (col < nn) { ex = nf + col; qu = Qw[ex]; }
+      } else if (col < Gmax + S) {
+        ex = s_se[q * S + col - Gmax];
+        qu = s_sq[q * S + col - Gmax];
+        if (ex >= 0) atomicAdd(&cnt_e[ex], 1);
+      } else {
+        ex = E;  // the shared-expert column
+      }
+      s_iex[q * G + col] = ex;
+      s_iqu[q * G + col] = qu;
+      s_rel[q * G + col] = run;
+      run += qu;
     }
   }
-  for (int i = tid; i < R * S; i += nthr)
-    if (s_se[i] >= 0) atomicAdd(&cnt_e[s_se[i]], 1);
-  if (warp == 0) {
-    // first row of each rank's block (routed rows only; a shared column moves it later)
-    int carry = 0;
+  if (warp == kSolveWarps - 1) {
+    // first row of each rank's block (routed rows only; a shared column moves
+    // it later), and the largest load before balancing
+    int carry = 0, bm = 0;
     for (int q0 = 0; q0 < R; q0 += 32) {
       const int q = q0 + lane;
       const int v = q < R ? s_Wf[q] : 0;
+      if (q < R) bm = max(bm, s_W0[q]);
       int incl = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -547,7 +541,11 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
       if (q < R) s_base[q] = carry + incl - v;
       carry += __shfl_sync(kFull, incl, 31);
     }
-    if (lane == 0) s_base[R] = carry;
+    bm = (int)__reduce_max_sync(kFull, (unsigned)bm);
+    if (lane == 0) {
+      s_base[R] = carry;
+      s_bmax = bm;
+    }
   }
   __syncthreads();
   // replica lists grouped by expert (CSR): the offsets rep_eptr and the list
@@ -571,23 +569,15 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   }
   if (lane == 31) s_wsum[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    const int v = lane < nthr / 32 ? s_wsum[lane] : 0;
-    int wi = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, wi, o);
-      if (lane >= o) wi += y;
-    }
-    if (lane < nthr / 32) s_wsum[lane] = wi - v;
-  }
-  __syncthreads();
+  int wbase = 0;  // the earlier warps' sums
+  for (int w = 0; w < warp; ++w) wbase += s_wsum[w];
 
   // ---- the global writes ----
   if (tid == 0) {
     ep_layer_stats* st = L.stats;
     st->status = hist_status | (s_any_cap ? EP_DEV_ITER_CAP : 0);
     s.acc_misc[0] = 0;  // zero again for the next call
+    s.acc_misc[2] = 0;
     st->before_max = s_bmax;
     st->cap_idx = s_best;
     st->stop_reason = s_wst[0];
@@ -604,7 +594,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
     L.W[q] = s_Wf[q];
     s.rank_rows[q] = s_Wf[q];  // routed rows per rank (the sampled mode recounts them)
   }
-  int run = s_wsum[warp] + incl - local;
+  int run = wbase + incl - local;
 #pragma unroll
   for (int u = 0; u < kIPT; ++u) {
     const int e = tid * kIPT + u;

@@ -660,6 +660,21 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   }
   pdl_wait();
   if (e >= d.E) return;
+  // Every load of the solve's tables that does not depend on another is
+  // issued first, together: the native's entry, the replica list's offset and
+  // the first 32 replica slots' entries (all slots for R*S <= 32).
+  const int h = home_of(e, E, R);
+  const int hcol = e - nat_first(h, E, R);
+  const int nat_rel = s.inst_rel[h * G + hcol], nat_q = L.inst_quota[h * G + hcol];
+  const int rep_off = L.rep_eptr[e];
+  bool hit0 = false;
+  int rel0 = 0, quota0 = 0;
+  if (lane < R * S) {
+    const int q = lane / S, col = d.Gmax + (lane - q * S);
+    hit0 = L.inst_expert[q * G + col] == e;
+    rel0 = s.inst_rel[q * G + col];
+    quota0 = L.inst_quota[q * G + col];
+  }
   int32_t* s_rb = s_rbw[warp];
   if (!d.sh && !d.sampled)  // issued now, read once the segments are written
     for (int q = lane; q <= d.R; q += 32) s_rb[q] = L.rank_base[q];
@@ -679,9 +694,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
       s.acc_load[r * E + e] = 0;  // zero again for the next call
     }
   }
-  const int h = home_of(e, E, R);
-  const int hcol = e - nat_first(h, E, R);
-  const int nat_rel = s.inst_rel[h * G + hcol], nat_q = L.inst_quota[h * G + hcol];
   for (int q = lane; q < R; q += 32) jof[q] = -1;
   __syncwarp();
   // instances in instance order: the replica slots holding e (scanned in slot
@@ -689,13 +701,13 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
   // after the replicas on ranks below h.  Every slot's entries are loaded in
   // one round, independent of each other.
   int nrep = 0, np = 0;
-  int32_t* rlist = L.rep_list + L.rep_eptr[e];  // e's part of the replica list
+  int32_t* rlist = L.rep_list + rep_off;  // e's part of the replica list
   for (int i0 = 0; i0 < R * S; i0 += 32) {
     const int i = i0 + lane;
     const int q = i / S, col = d.Gmax + (i - (i / S) * S);
-    bool hit = false;
-    int rel = 0, quota = 0;
-    if (i < R * S) {
+    bool hit = i0 == 0 && hit0;
+    int rel = i0 == 0 ? rel0 : 0, quota = i0 == 0 ? quota0 : 0;
+    if (i0 > 0 && i < R * S) {
       hit = L.inst_expert[q * G + col] == e;
       rel = s.inst_rel[q * G + col];
       quota = L.inst_quota[q * G + col];

@@ -200,6 +200,33 @@ def _timed(torch, fn, iters, stream, flush=None, skip=1):
     return out
 
 
+def _plan_back_to_back(torch, plan, ids, flush, stream, dev, n=50, reps=7):
+    """Device time per plan call when calls are queued back to back, as in a
+    step where the plan follows other GPU work: one CUDA graph of n times
+    [L2 flush, plan] against one of n L2 flushes alone, each replayed between
+    two events; (difference) / n, median of reps.  The single-call figures
+    above also hold the launch and event latency of an idle stream."""
+    g_stream = torch.cuda.Stream(device=dev)
+    g_stream.wait_stream(stream)
+    g_plan, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_plan, stream=g_stream):
+        for k in range(n):
+            flush.fill_(k & 0xFF)
+            plan.balance_layer(0, ids)
+    with torch.cuda.graph(g_flush, stream=g_stream):
+        for k in range(n):
+            flush.fill_(k & 0xFF)
+    stream.wait_stream(g_stream)
+    torch.cuda.synchronize()
+    per_call = []
+    for _ in range(reps):
+        t_plan = _timed(torch, g_plan.replay, 1, stream, skip=0)[0]
+        t_flush = _timed(torch, g_flush.replay, 1, stream, skip=0)[0]
+        per_call.append(1e3 * (t_plan - t_flush) / n)
+    del g_plan, g_flush
+    return {"median": _median(per_call), "calls_per_graph": n, "reps": reps}
+
+
 def _median(xs):
     xs = sorted(xs)
     return xs[len(xs) // 2]
@@ -336,8 +363,10 @@ def run_gpu(args):
                                             skip=3))
         plan_graph = {"median": _median(us), "mean": sum(us) / len(us), "iters": len(us)}
         del graph
+        plan_b2b = _plan_back_to_back(torch, plan, ids, flush, stream, dev)
     except RuntimeError as err:  # reported, not fatal: the eager figure stands
         plan_graph = {"error": str(err).splitlines()[0]}
+        plan_b2b = None
     stage_ms = _median(_timed(torch, lambda: plan.stage_replicas(0, native_w, slots), 5, stream, flush))
     reduce_ms = _median(_timed(torch, lambda: plan.reduce_replica_grads(0, slot_grads, native_grads),
                                5, stream, flush))
@@ -434,6 +463,7 @@ def run_gpu(args):
         "plan_us": {"median": _median(plan_us), "mean": sum(plan_us) / len(plan_us),
                     "p90": plan_us[int(len(plan_us) * 0.9)], "iters": len(plan_us)},
         "plan_us_cuda_graph": plan_graph,
+        "plan_us_back_to_back": plan_b2b,
         "permute_gbs": achieved,
         "stage_gbs": stage_bytes / (stage_ms * 1e-3) / 1e9 if n_rep else 0.0,
         "reduce_gbs": reduce_bytes / (reduce_ms * 1e-3) / 1e9 if n_rep else 0.0,

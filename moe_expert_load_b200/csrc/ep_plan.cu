@@ -859,20 +859,21 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) k_reroute(Dims d, LayerBu
     const int r = lane + 32 * k;
     if (r >= R) continue;
     int w = segbase[k];
-    // the record of (r, e) for the token assignment: {first segment's index in
-    // the lists, count | first rank << 16, first row base, second segment's
-    // first ordinal} and {second rank, second row base, third segment's first
-    // ordinal}; ordinals past the lists' end never occur
-    int4 r0 = make_int4(e * 3 * R + w, cnt[k], 0, INT_MAX);
-    int4 r1 = make_int4(0, 0, INT_MAX, 0);
+    // the record of (r, e) for the token assignment: {first row base
+    // (INT_MIN: no segment), second segment's first ordinal (INT_MAX: none),
+    // first rank, 0} and {second rank | segment count << 8, second row base,
+    // third segment's first ordinal (INT_MAX: none), index of the last
+    // segment in the lists}
+    int4 r0 = make_int4(INT_MIN, INT_MAX, 0, 0);
+    int4 r1 = make_int4(cnt[k] << 8, 0, INT_MAX, e * 3 * R + w + cnt[k] - 1);
     auto put = [&](int ord, int rank, int base) {
       const int i = w - segbase[k];
       if (i == 0) {
-        r0.y |= rank << 16;
-        r0.z = base;
+        r0.x = base;
+        r0.z = rank;
       } else if (i == 1) {
-        r0.w = ord;
-        r1.x = rank;
+        r0.y = ord;
+        r1.x |= rank;
         r1.y = base;
       } else if (i == 2) {
         r1.z = ord;
@@ -1044,8 +1045,10 @@ __host__ __device__ __forceinline__ bool assign_packed(const Dims& d) {
 
 template <int PASS>
 struct AssignCtx {
-  const int4* sge;       // [E+1] per-expert records of the first two segments (slot E: dummy)
-  const int4* rec1;      // [E] the second segment and where the third begins
+  const int2* sge;       // [E+1] per expert: first row base (INT_MIN: none), second
+                         // segment's first ordinal (slot E: dummy)
+  const uint8_t* rk0;    // [E+1] first segment's destination rank (PASS 1)
+  const int4* rec1;      // [E] second segment, where the third begins, last segment
   const int32_t* gord;   // the rerouting's segment lists in global memory
   const int32_t* gbase;
   const int32_t* grk;
@@ -1057,28 +1060,30 @@ struct AssignCtx {
 
 // The row (and destination rank) of ordinal o of expert e; ok is false for a
 // dropped id or an expert without segments.  The segment is the last one that
-// starts at or before o: the first two are in shared memory, a third or later
-// one (rare: a source rank's demand spread over several remote instances) is
-// found in the rerouting's list in global memory.
+// starts at or before o: the first two are in shared memory (the first in an
+// 8-byte record), a third or later one (rare: a source rank's demand spread
+// over several remote instances) is found in the rerouting's list in global
+// memory.
 template <int PASS>
 __device__ __forceinline__ void assign_finish(const AssignCtx<PASS>& c, int e, int o, bool valid,
                                               int idx, bool& inconsistent) {
-  const int4 g = c.sge[e];
-  const int n = g.y & 0xffff;
-  int b = g.z, q = g.y >> 16;
-  if (o >= g.w) {
+  const int2 g = c.sge[e];
+  int b = g.x, q = PASS > 0 ? c.rk0[e] : 0;
+  if (o >= g.y) {
     const int4 h = c.rec1[e];
     b = h.y;
-    q = h.x;
+    q = h.x & 0xff;
     if (o >= h.z) {
-      int si = g.x + n - 1;
-      while (si > g.x + 2 && c.gord[si] > o) --si;
+      const int third = h.w - (h.x >> 8) + 3;
+      int si = h.w;
+      while (si > third && c.gord[si] > o) --si;
       b = c.gbase[si];
       if (PASS > 0) q = c.grk[si];
     }
   }
-  const bool ok = valid && n > 0;
-  inconsistent |= valid && n == 0;
+  const bool has = g.x != INT_MIN;
+  const bool ok = valid && has;
+  inconsistent |= valid && !has;
   c.drow[idx] = ok ? b + o : -1;
   if (PASS > 0) {
     const uint8_t rank = ok ? (uint8_t)q : (uint8_t)kNoRank;
@@ -1146,9 +1151,10 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   // the rerouting's records of source rank r (see k_reroute); slot E of the
   // first table and of the running counts is a dummy that dropped ids (and
   // lanes past the end of the sub-chunk) share
-  int4* sge = reinterpret_cast<int4*>(sm);              // [E+1]
-  int4* rec1 = sge + E + 1;                             // [E]
-  int32_t* base0 = reinterpret_cast<int32_t*>(rec1 + E);  // [E]
+  int4* rec1 = reinterpret_cast<int4*>(sm);             // [E]
+  int2* sge = reinterpret_cast<int2*>(rec1 + E);        // [E+1]
+  uint8_t* rk0 = reinterpret_cast<uint8_t*>(sge + E + 1);  // [E+1] (PASS 1)
+  int32_t* base0 = sm + 4 * E + 2 * (E + 1) + (PASS > 0 ? (E + 4) / 4 : 0);  // [E]
   const int nsa = kPlanSubT * K;                        // assignments per sub-chunk
   const bool pk = assign_packed(d);                     // expert and ordinal in one word
   const int per_warp = E + 1 + nsa + (pk ? 0 : (nsa + 1) / 2) + (PASS > 0 ? R + (nsa + 3) / 4 : 0);
@@ -1222,9 +1228,14 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
     const int4* rec = reinterpret_cast<const int4*>(s.seg_rec) + (int64_t)r * E * 2;
     for (int i = tid; i < 2 * E; i += nthr) {
       const int4 x = rec[i];
-      if (i & 1) rec1[i >> 1] = x; else sge[i >> 1] = x;
+      if (i & 1) {
+        rec1[i >> 1] = x;
+      } else {
+        sge[i >> 1] = make_int2(x.x, x.y);
+        if (PASS > 0) rk0[i >> 1] = (uint8_t)x.z;
+      }
     }
-    if (tid == 0) sge[E] = make_int4(0, 1, 0, INT_MAX);
+    if (tid == 0) sge[E] = make_int2(0, INT_MAX);
   }
   if (PASS > 0)
     for (int q = tid; q < R; q += nthr) {
@@ -1237,7 +1248,7 @@ k_assign(const int32_t* __restrict__ ids, Dims d, LayerBuf L, Scratch s) {
   // Each assignment's ordinal selects its segment and thus its row: the
   // expert's segment record first (dropped ids share the dummy slot E).
   bool inconsistent = false;
-  AssignCtx<PASS> c{sge, rec1, s.seg_ord, s.seg_base, s.seg_rank, L.dst_row + rbase,
+  AssignCtx<PASS> c{sge, rk0, rec1, s.seg_ord, s.seg_base, s.seg_rank, L.dst_row + rbase,
                     PASS > 0 ? s.asg_rank + rbase : nullptr, dr, a0, E};
   __syncwarp();
 #pragma unroll 4
@@ -1898,7 +1909,8 @@ size_t assign_smem(const Dims& d, int pass) {
   const size_t nsa = (size_t)kPlanSubT * d.K;
   const size_t per_warp = (size_t)d.E + 1 + nsa + (assign_packed(d) ? 0 : (nsa + 1) / 2) +
                           (pass > 0 ? d.R + (nsa + 3) / 4 : 0);
-  return sizeof(int32_t) * (4 * ((size_t)d.E + 1) + 4 * (size_t)d.E + d.E +
+  return sizeof(int32_t) * (4 * (size_t)d.E + 2 * ((size_t)d.E + 1) +
+                            (pass > 0 ? ((size_t)d.E + 4) / 4 : 0) + d.E +
                             (size_t)kWarpsPerBlock * per_warp);
 }
 

@@ -262,30 +262,35 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
   // expert totals: the load matrix's columns summed over source ranks (the
   // histogram adds only into the load matrix: one total per expert would
   // take an atomic from every block of the grid).  CTA c of the cluster sums
-  // experts [c*E/n, (c+1)*E/n) — thread (slice, e) sums ranks slice,
-  // slice + nslice, ... of expert e, sixteen loads in flight — and every CTA
-  // then reads the other CTAs' totals from their shared memory.
+  // experts [c*E/n, (c+1)*E/n): nslice adjacent lanes (a power of two) share
+  // an expert, each summing ranks slice, slice + nslice, ... with sixteen
+  // loads in flight, and a shuffle reduction leaves the total with the
+  // group's first lane; every CTA then reads the other CTAs' totals from
+  // their shared memory.
   const int e_lo = crank * E / ncta, e_hi = (crank + 1) * E / ncta, ne = e_hi - e_lo;
-  for (int e = e_lo + tid; e < e_hi; e += nthr) Tot[e] = 0;
   for (int e = tid; e <= E; e += nthr) cnt_e[e] = 0;  // the winner's replica counts, at the end
   if (tid == 0) s_iter_cap_hit = 0;
-  __syncthreads();
   if (ne > 0) {
-    const int nslice = ne < nthr ? nthr / ne : 1;
-    for (int t = tid; t < nslice * ne; t += nthr) {
-      const int e = e_lo + t % ne, sl = t / ne;
+    int nslice = 1;
+    while (nslice < 32 && 2 * nslice * ne <= nthr) nslice *= 2;
+    for (int t0 = 0; t0 < nslice * ne; t0 += nthr) {  // warp-uniform rounds
+      const int t = t0 + tid;
+      const bool in = t < nslice * ne;
+      const int e = e_lo + t / nslice, sl = t % nslice;
       int acc = 0;
-      for (int r = sl; r < R; r += 16 * nslice) {
-        int v[16];
+      if (in)
+        for (int r = sl; r < R; r += 16 * nslice) {
+          int v[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int q = r + u * nslice;
-          v[u] = q < R ? s.acc_load[q * E + e] : 0;
+          for (int u = 0; u < 16; ++u) {
+            const int q = r + u * nslice;
+            v[u] = q < R ? s.acc_load[q * E + e] : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 16; ++u) acc += v[u];
         }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) acc += v[u];
-      }
-      if (acc) atomicAdd(&Tot[e], acc);
+      for (int o = nslice / 2; o > 0; o >>= 1) acc += __shfl_down_sync(kFull, acc, o, nslice);
+      if (in && sl == 0) Tot[e] = acc;
     }
   }
   cluster.sync();

@@ -223,7 +223,9 @@ __device__ __forceinline__ int warp_argmax_rank(const unsigned (&v)[RW], const b
 // registers; native quotas live in shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kSolveWarps = 4;                     // cap candidates per CTA: one per SM partition
-constexpr int kSolveThreads = kSolveWarps * 32;
+// plus as many helper warps, which wait at the barrier during the greedy and
+// halve the per-thread work of the setup and of the winner's table emit
+constexpr int kSolveThreads = 2 * kSolveWarps * 32;
 
 template <int SMAX, int RW, bool PACK>
 __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, Scratch s) {
@@ -314,7 +316,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
 
   // ---- one greedy run per warp: candidate j = crank * kSolveWarps + warp ----
   const int j = crank * kSolveWarps + warp;
-  const bool solver = j < d.J;
+  const bool solver = warp < kSolveWarps && j < d.J;
   const int64_t den = 200LL * R;
   const int C = (int)(((int64_t)A * (200 + j) + den - 1) / den);
   int Wr[RW], used[RW], se[RW][SMAX], sq[RW][SMAX];
@@ -529,7 +531,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1) k_solve(Dims d, LayerBuf L, 
       run += qu;
     }
   }
-  if (warp == kSolveWarps - 1) {
+  if (warp == kSolveThreads / 32 - 1) {  // a warp with no rank of its own above
     // first row of each rank's block (routed rows only; a shared column moves
     // it later), and the largest load before balancing
     int carry = 0, bm = 0;

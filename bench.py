@@ -363,7 +363,8 @@ def run_gpu(args):
                                             skip=3))
         plan_graph = {"median": _median(us), "mean": sum(us) / len(us), "iters": len(us)}
         del graph
-        plan_b2b = _plan_back_to_back(torch, plan, ids, flush, stream, dev)
+        plan_b2b = _plan_back_to_back(torch, plan, ids, flush, stream, dev,
+                                      reps=min(7, max(1, args.plan_iters)))
     except RuntimeError as err:  # reported, not fatal: the eager figure stands
         plan_graph = {"error": str(err).splitlines()[0]}
         plan_b2b = None

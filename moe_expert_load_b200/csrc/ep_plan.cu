@@ -210,8 +210,9 @@ __device__ __forceinline__ int warp_argmax_rank(const unsigned (&v)[RW], const b
 }
 
 // ---------------------------------------------------------------------------
-// a2: quota solve.  A thread-block cluster of ceil(J/4) CTAs of 4 warps, one
-// SM each; warp j of the cluster (CTA j/4) runs the greedy at cap
+// a2: quota solve.  A thread-block cluster of ceil(J/4) CTAs, one SM each;
+// cap-candidate warp j (warp j%4 of CTA j/4; warps 4-7 of every CTA help with
+// the setup and the table emit) runs the greedy at cap
 // C_j = ceil(A (200 + j) / (200 R)).  Greedy step: the most-loaded rank p that is
 // not stuck (smallest index on ties) gives min(max(W_p - C, m), slack_r, Q_e) of
 // its native e — natives tried by quota descending, then expert ascending, only

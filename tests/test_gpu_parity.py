@@ -685,6 +685,23 @@ def test_waterfill_standalone_parity(all_ranks):
             np.testing.assert_array_equal(count.cpu().numpy(), wc)
 
 
+def test_waterfill_hand_worked_draws_on_gpu():
+    # the hand-worked picks of tests/golden/waterfill_worked_draws.json, drawn
+    # by the device kernel (the expected values are the golden file's)
+    import json
+    import os
+
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "waterfill_worked_draws.json")))
+    load = np.array(g["load"], dtype=np.int32)
+    for d in g["draws"]:
+        dst = np.full((g["R"], g["T"], g["K"]), -1, np.int32)
+        dst[d["r"], 0] = d["routes"]
+        pick, _ = ep_waterfill(torch.from_numpy(load).cuda(), torch.from_numpy(dst).cuda(),
+                               seed=int(d["seed"]), bonus_permille=d["bonus_permille"])
+        torch.cuda.synchronize()
+        assert int(pick.cpu().numpy()[d["r"], 0]) == d["pick"], d
+
+
 @pytest.mark.parametrize("name,all_ranks,sampled", [
     ("dsv3", False, False), ("tiny", True, False), ("dsv3", False, True)])
 def test_waterfill_layer_rerun_equals_a_fresh_balance(name, all_ranks, sampled):

@@ -319,6 +319,22 @@ def test_waterfill_all_slack_on_one_candidate():
     assert cnt.sum() == R * T
 
 
+def test_waterfill_hand_worked_draws():
+    # three picks worked by hand from the published SplitMix64 vector
+    # (tests/golden/waterfill_worked_draws.json): a draw on an interval
+    # boundary, the first of the other candidates, and the local preference
+    g = json.load(open(os.path.join(GOLDEN, "waterfill_worked_draws.json")))
+    load = np.array(g["load"])
+    H, B0, slack = oracle.waterline(load, g["R"] * g["T"], 0)
+    assert H == 8 and B0 == 0 and slack.tolist() == [0, 2, 6, 0]
+    for d in g["draws"]:
+        dst = np.full((g["R"], g["T"], g["K"]), -1, np.int32)
+        dst[d["r"], 0] = d["routes"]
+        pick, cnt = oracle.waterfill(load, dst, seed=int(d["seed"]), bonus_permille=d["bonus_permille"])
+        assert int(pick[d["r"], 0]) == d["pick"], d
+        assert cnt.sum() == g["R"] * g["T"]
+
+
 def test_waterfill_fallback_prefers_clearly_lighter():
     # loads [12, 10, 10, 0] with N = 4: H = ceil(36/4) = 9, no slack on ranks 0..2.
     # Token on rank 0 visiting rank 1 only: candidates {0, 1}, min load 10 on rank 1.
